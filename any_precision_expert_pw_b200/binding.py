@@ -1,0 +1,162 @@
+"""ctypes binding of libpw (include/pw.h): the same entry points, same names, same arguments.
+
+Pointers are passed as Python ints (device addresses, e.g. ``tensor.data_ptr()``) and streams as
+raw ``cudaStream_t`` values (``torch.cuda.current_stream().cuda_stream``).  Every function
+returns the ``pw_status`` code as an int; ``check()`` turns a non-zero code into ``PwError``.
+There is no fallback: if ``libpw.so`` is missing the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libpw.so")
+
+PW_OK = 0
+PW_ERR_INVALID_ARG = 1
+PW_ERR_UNSUPPORTED = 2
+PW_ERR_CUDA = 3
+PW_ERR_NOT_RESIDENT = 4
+PW_ERR_TIMEOUT = 5
+PW_ERR_BAD_EXPERT = 6
+PW_ERR_BAD_BITS = 7
+
+PW_MOD_GATE_UP = 0
+PW_MOD_DOWN = 1
+PW_PAGE_GPU, PW_PAGE_CPU, PW_PAGE_XFER = 0, 1, 2
+PW_POLICY_FETCH_ALL, PW_POLICY_THRESHOLD, PW_POLICY_FIRST_CHOICE = 0, 1, 2
+PW_ACT_HIT, PW_ACT_FETCH, PW_ACT_SUBST = 0, 1, 2
+PW_MIN_BITS = 3
+PW_MAX_BITS = 8
+PW_MAX_EXPERTS = 1024
+PW_MAX_TOPK = 16
+PW_MAX_TOKENS = 4096
+
+# every symbol include/pw.h declares
+EXPORTS = ("pw_block_prepare", "pw_pack_bitplanes", "pw_route_topk", "pw_substitute",
+           "pw_remap", "pw_moe_workspace_bytes", "pw_moe_anyprec_forward", "pw_commit_bits",
+           "pw_get_status", "pw_status_string", "pw_version")
+
+
+class PwError(RuntimeError):
+    def __init__(self, code: int, where: str = ""):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)} ({code})")
+
+
+class pw_block(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_uint32), ("cols", ctypes.c_uint32),
+                ("parent_bits", ctypes.c_uint8), ("min_bits", ctypes.c_uint8),
+                ("desired_bits", ctypes.c_uint8), ("committed_bits", ctypes.c_uint8),
+                ("state", ctypes.c_uint8), ("reserved0", ctypes.c_uint8 * 3),
+                ("planes", ctypes.c_void_p), ("lut", ctypes.c_void_p * 9),
+                ("reserved1", ctypes.c_uint8 * 32), ("tma_desc", ctypes.c_uint8 * 128)]
+
+
+class pw_page_table(ctypes.Structure):
+    _fields_ = [("num_layers", ctypes.c_uint32), ("num_experts", ctypes.c_uint32),
+                ("blocks", ctypes.c_void_p)]
+
+
+class pw_route_cfg(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_int32), ("renorm", ctypes.c_int32), ("policy", ctypes.c_int32),
+                ("threshold", ctypes.c_float), ("critical_n", ctypes.c_int32)]
+
+
+assert ctypes.sizeof(pw_block) == 256 and pw_block.tma_desc.offset == 128
+assert ctypes.sizeof(pw_page_table) == 16 and ctypes.sizeof(pw_route_cfg) == 20
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libpw.so (built in-tree); raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libpw.so not found at {LIB_PATH}; build it first "
+                               "(python -c 'import __graft_entry__ as g; g.build()')")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, Z, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
+        L.pw_block_prepare.argtypes = [ctypes.POINTER(pw_block)]
+        L.pw_pack_bitplanes.argtypes = [P, I, I, I, P, S]
+        L.pw_route_topk.argtypes = [P, P, P, I, I, I, ctypes.POINTER(pw_route_cfg), P, P, P, S]
+        L.pw_substitute.argtypes = [P, P, P, P, I, I, ctypes.POINTER(pw_route_cfg), P, P, S]
+        L.pw_remap.argtypes = [P, P, P, I, I, ctypes.POINTER(pw_route_cfg), P, S]
+        L.pw_moe_workspace_bytes.argtypes = [I, I, I, I, I]
+        L.pw_moe_workspace_bytes.restype = Z
+        L.pw_moe_anyprec_forward.argtypes = [P, I, I, P, I, I, I, I, P, P, P, P, Z, S]
+        L.pw_commit_bits.argtypes = [P, I, P, P, I, S]
+        L.pw_get_status.argtypes = [S]
+        L.pw_status_string.argtypes = [I]
+        L.pw_status_string.restype = ctypes.c_char_p
+        L.pw_version.restype = ctypes.c_char_p
+        for name in EXPORTS:
+            fn = getattr(L, name)
+            if name not in ("pw_moe_workspace_bytes", "pw_status_string", "pw_version"):
+                fn.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    try:
+        return lib().pw_status_string(int(code)).decode()
+    except Exception:  # library missing: still give a readable error
+        return f"status {code}"
+
+
+def check(code: int, where: str = "libpw") -> None:
+    if code != PW_OK:
+        raise PwError(code, where)
+
+
+def _cfg(cfg):
+    return ctypes.byref(cfg) if cfg is not None else None
+
+
+def pw_version() -> str:
+    return lib().pw_version().decode()
+
+
+def pw_status_string(code: int) -> str:
+    return lib().pw_status_string(int(code)).decode()
+
+
+def pw_block_prepare(blk: pw_block) -> int:
+    return lib().pw_block_prepare(ctypes.byref(blk))
+
+
+def pw_pack_bitplanes(idx, rows, cols, n, planes, stream=0) -> int:
+    return lib().pw_pack_bitplanes(idx, rows, cols, n, planes, stream)
+
+
+def pw_route_topk(x_bf16, Wr, bias, T, H, E, cfg, logits, idx, gate, stream=0) -> int:
+    return lib().pw_route_topk(x_bf16, Wr, bias, T, H, E, _cfg(cfg), logits, idx, gate, stream)
+
+
+def pw_substitute(logits, idx, gate, resident, T, E, cfg, action, mass, stream=0) -> int:
+    return lib().pw_substitute(logits, idx, gate, resident, T, E, _cfg(cfg), action, mass, stream)
+
+
+def pw_remap(logits, idx, gate, T, E, cfg, critical, stream=0) -> int:
+    return lib().pw_remap(logits, idx, gate, T, E, _cfg(cfg), critical, stream)
+
+
+def pw_moe_workspace_bytes(T, k, E, H, I) -> int:
+    return int(lib().pw_moe_workspace_bytes(T, k, E, H, I))
+
+
+def pw_moe_anyprec_forward(pt_dev, layer, E, x_bf16, T, H, I, k, idx, gate, y, workspace,
+                           ws_bytes, stream=0) -> int:
+    return lib().pw_moe_anyprec_forward(pt_dev, layer, E, x_bf16, T, H, I, k, idx, gate, y,
+                                        workspace, ws_bytes, stream)
+
+
+def pw_commit_bits(pt_dev, num_blocks, block_ids, q, count, stream=0) -> int:
+    return lib().pw_commit_bits(pt_dev, num_blocks, block_ids, q, count, stream)
+
+
+def pw_get_status(stream=0) -> int:
+    return lib().pw_get_status(stream)

@@ -1,0 +1,334 @@
+// libpw: host side of the C ABI declared in include/pw.h.  One translation unit: the step
+// kernels live in the pw_*.cuh headers included below.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "pw.h"
+#include "pw_common.cuh"
+#include "pw_ffn.cuh"
+#include "pw_group.cuh"
+#include "pw_pack.cuh"
+#include "pw_route.cuh"
+#include "pw_table.cuh"
+
+static_assert(sizeof(pw_block) == 256, "pw_block layout");
+static_assert(offsetof(pw_block, planes) == 16, "pw_block layout");
+static_assert(offsetof(pw_block, lut) == 24, "pw_block layout");
+static_assert(offsetof(pw_block, tma_desc) == 128, "pw_block layout");
+static_assert(sizeof(CUtensorMap) == 128, "tensor map size");
+static_assert(sizeof(pw_page_table) == 16, "pw_page_table layout");
+static_assert(sizeof(pw_route_cfg) == 20, "pw_route_cfg layout");
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+inline cudaStream_t as_cuda(pw_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline pw_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? PW_OK : PW_ERR_CUDA;
+}
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct DeviceInfo {
+  int sms = 0;
+  bool ffn_attr_set = false;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+// Per-device, once: SM count and the large dynamic shared memory opt-in of the FFN kernels.
+pw_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PW_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (d.sms == 0) {
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return PW_ERR_CUDA;
+  }
+  if (!d.ffn_attr_set) {
+    if (cudaFuncSetAttribute(pw::k4::ffn_kernel<pw::k4::MODE_GATE_UP>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             pw::k4::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(pw::k4::ffn_kernel<pw::k4::MODE_DOWN>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             pw::k4::kSmemBytes) != cudaSuccess)
+      return PW_ERR_CUDA;
+    d.ffn_attr_set = true;
+  }
+  *out = &d;
+  return PW_OK;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) ==
+            cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Workspace layout of pw_moe_anyprec_forward.
+struct Workspace {
+  size_t counts, offsets, perm, inv, active, meta, X, Hbuf, O, total;
+  int ldx, ldh;
+};
+
+Workspace ws_layout(int T, int k, int E, int H, int I) {
+  Workspace w;
+  const size_t TK = static_cast<size_t>(T) * k;
+  w.ldx = static_cast<int>(align_up(H, pw::k4::kStageCols));
+  w.ldh = static_cast<int>(align_up(I, pw::k4::kStageCols));
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align_up(o + bytes, 256);
+    return at;
+  };
+  w.counts = take(4 * static_cast<size_t>(E));
+  w.offsets = take(4 * static_cast<size_t>(E + 1));
+  w.perm = take(4 * TK);
+  w.inv = take(4 * TK);
+  w.active = take(4 * static_cast<size_t>(E));
+  w.meta = take(16);
+  w.X = take(4 * TK * w.ldx);
+  w.Hbuf = take(4 * TK * w.ldh);
+  w.O = take(4 * TK * H);
+  w.total = o;
+  return w;
+}
+
+bool cfg_ok(const pw_route_cfg* cfg, int E) {
+  return cfg && cfg->k >= 1 && cfg->k <= PW_MAX_TOPK && cfg->k <= E;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pw_version(void) { return "libpw 0.1 (sm_100a)"; }
+
+const char* pw_status_string(pw_status s) {
+  switch (s) {
+    case PW_OK: return "PW_OK";
+    case PW_ERR_INVALID_ARG: return "PW_ERR_INVALID_ARG";
+    case PW_ERR_UNSUPPORTED: return "PW_ERR_UNSUPPORTED";
+    case PW_ERR_CUDA: return "PW_ERR_CUDA";
+    case PW_ERR_NOT_RESIDENT: return "PW_ERR_NOT_RESIDENT";
+    case PW_ERR_TIMEOUT: return "PW_ERR_TIMEOUT";
+    case PW_ERR_BAD_EXPERT: return "PW_ERR_BAD_EXPERT";
+    case PW_ERR_BAD_BITS: return "PW_ERR_BAD_BITS";
+  }
+  return "PW_ERR_UNKNOWN";
+}
+
+pw_status pw_block_prepare(pw_block* blk) {
+  if (!blk || !blk->planes) return PW_ERR_INVALID_ARG;
+  const uint32_t rows = blk->rows, cols = blk->cols;
+  const int n = blk->parent_bits, mn = blk->min_bits;
+  if (rows == 0 || cols == 0 || rows % 32 || cols % 128) return PW_ERR_INVALID_ARG;
+  if (n < 1 || n > PW_MAX_BITS || mn < 1 || mn > n) return PW_ERR_INVALID_ARG;
+  if (static_cast<uint64_t>(rows) * n > 0x7fffffffull) return PW_ERR_UNSUPPORTED;
+  if (reinterpret_cast<uintptr_t>(blk->planes) % 16) return PW_ERR_INVALID_ARG;
+  for (int b = 0; b <= PW_MAX_BITS; ++b) {
+    const bool want = (b >= mn && b <= n);
+    if (want && (!blk->lut[b] || reinterpret_cast<uintptr_t>(blk->lut[b]) % 16))
+      return PW_ERR_INVALID_ARG;
+  }
+  if (blk->committed_bits < mn || blk->committed_bits > n) return PW_ERR_INVALID_ARG;
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return PW_ERR_CUDA;
+  // planes viewed as a 2-D uint32 tensor [n * rows][cols / 32]; box = 32 words x 16 rows
+  const cuuint64_t dims[2] = {cols / 32u, static_cast<cuuint64_t>(rows) * n};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols / 32u) * 4u};
+  const cuuint32_t box[2] = {pw::k4::kStageWords, pw::k4::kSegRows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUtensorMap map;
+  memset(&map, 0, sizeof(map));
+  const CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2,
+                         const_cast<uint32_t*>(blk->planes), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return PW_ERR_CUDA;
+  memcpy(blk->tma_desc, &map, sizeof(map));
+  return PW_OK;
+}
+
+pw_status pw_pack_bitplanes(const uint8_t* idx, int rows, int cols, int n, uint32_t* planes,
+                            pw_stream_t stream) {
+  if (!idx || !planes || rows <= 0 || cols <= 0 || cols % 32 || n < 1 || n > 8)
+    return PW_ERR_INVALID_ARG;
+  const long long words = static_cast<long long>(rows) * (cols / 32);
+  const long long blocks = (words + 7) / 8;
+  const int grid = static_cast<int>(blocks < 65535LL * 16 ? blocks : 65535LL * 16);
+  pw::pack_bitplanes_kernel<<<grid, 256, 0, as_cuda(stream)>>>(idx, rows, cols, n, planes);
+  return launch_status();
+}
+
+pw_status pw_route_topk(const uint16_t* x_bf16, const float* Wr, const float* bias, int T, int H,
+                        int E, const pw_route_cfg* cfg, float* logits, int32_t* idx, float* gate,
+                        pw_stream_t stream) {
+  if (!x_bf16 || !Wr || !logits || !idx || !gate) return PW_ERR_INVALID_ARG;
+  if (T < 1 || T > PW_MAX_TOKENS || E < 1 || E > PW_MAX_EXPERTS || H < 1 || !cfg_ok(cfg, E))
+    return PW_ERR_INVALID_ARG;
+  const dim3 g1((E + pw::kRouteExpertsPerCta - 1) / pw::kRouteExpertsPerCta,
+                (T + pw::kRouteTokensPerCta - 1) / pw::kRouteTokensPerCta);
+  pw::router_logits_kernel<<<g1, 256, 0, as_cuda(stream)>>>(x_bf16, Wr, bias, T, H, E, logits);
+  if (launch_status() != PW_OK) return PW_ERR_CUDA;
+  pw::topk_kernel<<<(T + 7) / 8, 256, 0, as_cuda(stream)>>>(logits, T, E, cfg->k, cfg->renorm,
+                                                            idx, gate);
+  return launch_status();
+}
+
+pw_status pw_substitute(const float* logits, int32_t* idx, const float* gate,
+                        const uint8_t* resident, int T, int E, const pw_route_cfg* cfg,
+                        uint8_t* action, float* mass, pw_stream_t stream) {
+  if (!logits || !idx || !gate || !resident) return PW_ERR_INVALID_ARG;
+  if (T < 1 || T > PW_MAX_TOKENS || E < 1 || E > PW_MAX_EXPERTS || !cfg_ok(cfg, E))
+    return PW_ERR_INVALID_ARG;
+  if (cfg->policy != PW_POLICY_FETCH_ALL && cfg->policy != PW_POLICY_THRESHOLD &&
+      cfg->policy != PW_POLICY_FIRST_CHOICE)
+    return PW_ERR_INVALID_ARG;
+  if (cfg->threshold != cfg->threshold) return PW_ERR_INVALID_ARG;  // NaN
+  pw::substitute_kernel<<<(T + 7) / 8, 256, 0, as_cuda(stream)>>>(
+      logits, idx, gate, resident, T, E, cfg->k, cfg->policy, cfg->threshold, action, mass);
+  return launch_status();
+}
+
+pw_status pw_remap(const float* logits, int32_t* idx, const float* gate, int T, int E,
+                   const pw_route_cfg* cfg, uint8_t* critical, pw_stream_t stream) {
+  if (!logits || !idx || !gate) return PW_ERR_INVALID_ARG;
+  if (T < 1 || T > PW_MAX_TOKENS || E < 1 || E > PW_MAX_EXPERTS || !cfg_ok(cfg, E))
+    return PW_ERR_INVALID_ARG;
+  if (cfg->critical_n < 0 || static_cast<long long>(T) * cfg->k > 8192) return PW_ERR_INVALID_ARG;
+  pw::remap_kernel<<<1, 1024, 0, as_cuda(stream)>>>(logits, idx, gate, T, E, cfg->k,
+                                                    cfg->critical_n, critical);
+  return launch_status();
+}
+
+size_t pw_moe_workspace_bytes(int T, int k, int E, int H, int I) {
+  if (T < 1 || k < 1 || E < 1 || H < 1 || I < 1) return 0;
+  return ws_layout(T, k, E, H, I).total;
+}
+
+pw_status pw_moe_anyprec_forward(const pw_page_table* pt_dev, int layer, int E,
+                                 const uint16_t* x_bf16, int T, int H, int I, int k,
+                                 const int32_t* idx, const float* gate, float* y, void* workspace,
+                                 size_t ws_bytes, pw_stream_t stream) {
+  if (!pt_dev || !x_bf16 || !idx || !gate || !y || !workspace) return PW_ERR_INVALID_ARG;
+  if (T < 1 || T > PW_MAX_TOKENS || k < 1 || k > PW_MAX_TOPK || layer < 0) return PW_ERR_INVALID_ARG;
+  if (E < 1 || E > PW_MAX_EXPERTS || k > E) return PW_ERR_INVALID_ARG;
+  if (H < 128 || I < 128 || H % 128 || I % 128) return PW_ERR_INVALID_ARG;
+  if (static_cast<long long>(T) * k > pw::kMaxAssign) return PW_ERR_UNSUPPORTED;
+  if (reinterpret_cast<uintptr_t>(workspace) % 256) return PW_ERR_INVALID_ARG;
+  const Workspace w = ws_layout(T, k, E, H, I);
+  if (ws_bytes < w.total) return PW_ERR_INVALID_ARG;
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != PW_OK) return PW_ERR_CUDA;
+  cudaStream_t st = as_cuda(stream);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  int32_t* counts = reinterpret_cast<int32_t*>(base + w.counts);
+  int32_t* offsets = reinterpret_cast<int32_t*>(base + w.offsets);
+  int32_t* perm = reinterpret_cast<int32_t*>(base + w.perm);
+  int32_t* inv = reinterpret_cast<int32_t*>(base + w.inv);
+  int32_t* active = reinterpret_cast<int32_t*>(base + w.active);
+  int32_t* meta = reinterpret_cast<int32_t*>(base + w.meta);
+  float* X = reinterpret_cast<float*>(base + w.X);
+  float* Hb = reinterpret_cast<float*>(base + w.Hbuf);
+  float* O = reinterpret_cast<float*>(base + w.O);
+  const int TK = T * k;
+
+  pw::group_kernel<<<1, pw::kGroupThreads, 0, st>>>(idx, TK, E, counts, offsets, perm, inv,
+                                                     active, meta);
+  if (launch_status() != PW_OK) return PW_ERR_CUDA;
+  pw::check_table_kernel<<<1, 32, 0, st>>>(pt_dev, layer, E, meta);
+  if (launch_status() != PW_OK) return PW_ERR_CUDA;
+  {
+    const dim3 g((w.ldx + 255) / 256, TK);
+    pw::prep_kernel<<<g, 256, 0, st>>>(x_bf16, perm, meta, k, H, w.ldx, X, I, w.ldh, Hb);
+    if (launch_status() != PW_OK) return PW_ERR_CUDA;
+  }
+  const int max_active = E < TK ? E : TK;
+  pw::k4::Params p;
+  p.pt = pt_dev;
+  p.layer = layer;
+  p.E = E;
+  p.counts = counts;
+  p.offsets = offsets;
+  p.active = active;
+  p.meta = meta;
+  // gate_up: h = SiLU(W_gate x) * (W_up x)
+  p.rows = 2 * I;
+  p.cols = H;
+  p.half = I;
+  p.tiles = I / pw::k4::kSegRows;
+  p.act = X;
+  p.ld_act = w.ldx;
+  p.out = Hb;
+  p.ld_out = w.ldh;
+  {
+    const long long items = static_cast<long long>(max_active) * p.tiles;
+    const int grid = static_cast<int>(items < di->sms ? items : di->sms);
+    pw::k4::ffn_kernel<pw::k4::MODE_GATE_UP>
+        <<<grid, pw::k4::kThreads, pw::k4::kSmemBytes, st>>>(p);
+    if (launch_status() != PW_OK) return PW_ERR_CUDA;
+  }
+  // down: o = W_down h
+  p.rows = H;
+  p.cols = I;
+  p.half = 0;
+  p.tiles = H / pw::k4::kRows;
+  p.act = Hb;
+  p.ld_act = w.ldh;
+  p.out = O;
+  p.ld_out = H;
+  {
+    const long long items = static_cast<long long>(max_active) * p.tiles;
+    const int grid = static_cast<int>(items < di->sms ? items : di->sms);
+    pw::k4::ffn_kernel<pw::k4::MODE_DOWN><<<grid, pw::k4::kThreads, pw::k4::kSmemBytes, st>>>(p);
+    if (launch_status() != PW_OK) return PW_ERR_CUDA;
+  }
+  {
+    const dim3 g((H + 255) / 256, T);
+    pw::combine_kernel<<<g, 256, 0, st>>>(O, inv, gate, meta, T, k, H, y);
+  }
+  return launch_status();
+}
+
+pw_status pw_commit_bits(pw_page_table* pt_dev, int num_blocks, const int32_t* block_ids,
+                         const uint8_t* q, int count, pw_stream_t stream) {
+  if (!pt_dev || !block_ids || !q || count < 0 || num_blocks < 1) return PW_ERR_INVALID_ARG;
+  if (count == 0) return PW_OK;
+  pw::commit_bits_kernel<<<(count + 255) / 256, 256, 0, as_cuda(stream)>>>(pt_dev, num_blocks,
+                                                                           block_ids, q, count);
+  return launch_status();
+}
+
+pw_status pw_get_status(pw_stream_t stream) {
+  if (cudaStreamSynchronize(as_cuda(stream)) != cudaSuccess) return PW_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, pw::g_status, sizeof(int)) != cudaSuccess) return PW_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(pw::g_status, &zero, sizeof(int)) != cudaSuccess) return PW_ERR_CUDA;
+  return static_cast<pw_status>(v);
+}
+
+}  // extern "C"

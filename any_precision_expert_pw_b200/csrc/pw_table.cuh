@@ -1,0 +1,44 @@
+// Weight Page Table kernels (PagedWeight, "Composants Clés" 1 and 3): stream-ordered commits of
+// q_i, so a commit lands exactly between two forward calls (a safe boundary), and the per-call
+// check of the table against the caller's layer and expert count.
+#pragma once
+#include "pw_common.cuh"
+
+namespace pw {
+
+__global__ void commit_bits_kernel(pw_page_table* __restrict__ pt, int num_blocks,
+                                   const int32_t* __restrict__ ids, const uint8_t* __restrict__ q,
+                                   int count) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= count) return;
+  const long long table_blocks = static_cast<long long>(pt->num_layers) * pt->num_experts * 2;
+  const int bid = ids[i];
+  if (bid < 0 || bid >= num_blocks || bid >= table_blocks) {
+    set_status(PW_ERR_BAD_BITS);
+    return;
+  }
+  pw_block* b = pt->blocks + bid;
+  const int qq = q[i];
+  if (qq < b->min_bits || qq > b->parent_bits || qq < 1 || qq > PW_MAX_BITS ||
+      b->lut[qq] == nullptr) {
+    set_status(PW_ERR_BAD_BITS);
+    return;
+  }
+  b->committed_bits = static_cast<uint8_t>(qq);
+}
+
+// meta[2] = 1 (and no active experts) when the table does not match (layer, E).
+__global__ void check_table_kernel(const pw_page_table* __restrict__ pt, int layer, int E,
+                                   int32_t* __restrict__ meta) {
+  if (threadIdx.x != 0) return;
+  const bool bad = pt->blocks == nullptr || static_cast<unsigned>(layer) >= pt->num_layers ||
+                   static_cast<int>(pt->num_experts) != E ||
+                   (reinterpret_cast<uintptr_t>(pt->blocks) & 63) != 0;
+  if (bad) {
+    set_status(PW_ERR_INVALID_ARG);
+    meta[0] = 0;
+  }
+  meta[2] = bad ? 1 : 0;
+}
+
+}  // namespace pw

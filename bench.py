@@ -1,0 +1,408 @@
+#!/usr/bin/env python
+"""Benchmark of the any-precision MoE decode layer (one JSON line on rank 0).
+
+Default workload: the Mixtral-8x7B-shaped layer (H 4096, 8 experts, I 14336, top-2 renormalised,
+parent 8-bit, per-block bitwidth uniform in 3..8, Zipf(1.2) router bias) at batch 1, synthetic
+seeded data.  A step is one whole layer call: router GEMV + softmax top-k (+ the config's
+substitution or remap) + grouping + fused any-precision FFN + combine, replayed from a CUDA
+graph.  L2 is flushed (a memset of 2.5x the L2 size) before every timed step, outside that
+step's CUDA events.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl pw|reference]
+
+N > 1 runs N independent replicas (one per GPU, launched by torchrun); value = N * T / (max over
+ranks of the per-step device time).  --impl reference times the CPU oracle on rank 0 instead.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE decode layer tokens/s and effective weight HBM GB/s (fraction of peak)"
+FALLBACK_HBM_GBS = 6650.0
+WORKLOAD = ("mixtral_8x7b", 1)
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=("pw", "reference"), default="pw")
+    ap.add_argument("--workload", default=f"{WORKLOAD[0]}:{WORKLOAD[1]}",
+                    help="config name:T (default mixtral_8x7b:1)")
+    ap.add_argument("--cpu-sample-rows", type=float, default=None,
+                    help="fraction of FFN rows the CPU oracle sample computes")
+    return ap.parse_args()
+
+
+def workload(args):
+    from any_precision_expert_pw_b200.inputs import CONFIGS
+    name, T = args.workload.split(":")
+    return CONFIGS[name], int(T)
+
+
+def read_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "any_precision_expert_pw_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM traffic per FFN call from the committed ncu summary, if it matches this source."""
+    p = os.path.join(ROOT, "profiles", "ffn_traffic.txt")
+    try:
+        kv = {}
+        for line in open(p):
+            if "=" in line and not line.startswith("#"):
+                k, v = line.strip().split("=", 1)
+                kv[k.strip()] = v.strip()
+        if kv.get("source_sha") == kernel_source_hash():
+            return float(kv["traffic_bytes_per_call"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", self.gpu_id], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sms, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sms.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sms) if sms else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sms)}
+
+
+def dist_init(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device(f"cuda:{local}"))
+    return world, rank, local
+
+
+def oracle_step(L, frac):
+    """One bounded oracle sample: full routing, FFN on a fraction of every block's rows.
+    Returns the seconds a full step would take (FFN time scaled by 1/frac)."""
+    import numpy as np
+    from oracle import ffn as offn
+    from oracle import layer as olayer
+    from oracle.group import group_by_expert
+    from oracle.router import bf16_bits_to_f64
+    cfg = L.cfg
+    if frac >= 1.0:                       # the whole layer, exactly as the oracle computes it
+        t0 = time.perf_counter()
+        olayer.moe_layer(L)
+        return time.perf_counter() - t0
+    t0 = time.perf_counter()
+    res = olayer.route(L)
+    t1 = time.perf_counter()
+    idx = res["idx"]
+    X = bf16_bits_to_f64(L.x_bf16)
+    _, offsets, perm, active = group_by_expert(idx, cfg.E)
+    rg = max(1, int(round(2 * cfg.I * frac)))
+    rd = max(1, int(round(cfg.H * frac)))
+    for e in active:
+        a = perm[offsets[e]:offsets[e + 1]]
+        Xe = X[a // cfg.k]
+        qg, qd = int(L.q[e, 0]), int(L.q[e, 1])
+        gu = offn.block_matvec(L.idx[e][0][:rg], L.lut[e][0][qg][:rg], cfg.n, qg, Xe.T)
+        h = np.zeros((cfg.I, len(a)))
+        h[: min(rg, cfg.I)] = gu[: min(rg, cfg.I)]
+        offn.block_matvec(L.idx[e][1][:rd], L.lut[e][1][qd][:rd], cfg.n, qd, h)
+    t2 = time.perf_counter()
+    return (t1 - t0) + (t2 - t1) / frac
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 1) for d in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(L, T, frac, reps=1):
+    secs = [oracle_step(L, frac) for _ in range(reps)]
+    s = statistics.median(secs)
+    return {"value": T / s, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": (f"float64 NumPy oracle, whole layer (routing + FFN + combine) on the "
+                       f"bench inputs; median of {reps}" if frac >= 1.0 else
+                       f"float64 NumPy oracle: full routing + FFN over {frac:.3f} of every used "
+                       f"block's rows, time scaled to the whole layer; median of {reps}")}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from any_precision_expert_pw_b200.inputs import make_layer
+    cfg, T = workload(args)
+    L = make_layer(cfg, T)
+    frac = args.cpu_sample_rows or 1.0
+    steps = max(1, min(args.steps, 10))
+    warm = max(0, min(args.warmup, 1))
+    for _ in range(warm):
+        oracle_step(L, frac)
+    secs = [oracle_step(L, frac) for _ in range(steps)]
+    s = sum(secs) / len(secs)
+    v = T / s
+    out = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
+           "n_gpus": world, "steps": steps, "warmup": warm, "ms_per_step": s * 1e3,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic",
+           "config": {"workload": f"{cfg.name}-shaped MoE decode layer, T={T}", "H": cfg.H,
+                      "E": cfg.E, "I": cfg.I, "k": cfg.k, "parent_bits": cfg.n},
+           "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": blas_threads(),
+                            "kind": "oracle",
+                            "sample": f"FFN over {frac:.3f} of every used block's rows per step, "
+                                      "time scaled to the whole layer"},
+           "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def run_pw(args):
+    import numpy as np
+    import torch
+
+    from any_precision_expert_pw_b200 import binding as B
+    from any_precision_expert_pw_b200.accounting import ffn_bytes, layer_bytes
+    from any_precision_expert_pw_b200.device_layer import DeviceLayer
+    from any_precision_expert_pw_b200.inputs import POLICY_NONE, make_layer
+
+    world, rank, local = dist_init(args.gpus)
+    dev = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(dev)
+    cfg, T = workload(args)
+    L = make_layer(cfg, T)
+    D = DeviceLayer(L, device=str(dev))
+    stream = torch.cuda.Stream(device=dev)
+    D.stream = stream.cuda_stream
+    with torch.cuda.stream(stream):
+        D.forward()
+    stream.synchronize()
+    st = D.status()
+    if st != B.PW_OK:
+        raise RuntimeError(f"device status after warm-up: {B.pw_status_string(st)}")
+
+    # parity of this run's routing against the oracle (cheap part of the check)
+    if rank == 0:
+        from oracle.layer import route as oracle_route
+        ref = oracle_route(L)
+        if not np.array_equal(D.idx.cpu().numpy(), ref["idx"]):
+            raise RuntimeError("routing of the bench inputs differs from the oracle")
+
+    g_step = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step, stream=stream):
+        D.forward()
+    g_ffn = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_ffn, stream=stream):
+        D.ffn()
+    launches_step = 2 + (0 if cfg.policy == POLICY_NONE else 1) + 6
+
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(int(2.5 * l2), dtype=torch.uint8, device=dev)
+
+    def timed(graph, n, record=True):
+        evs = []
+        with torch.cuda.stream(stream):
+            for _ in range(n):
+                flush.fill_(1)
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                graph.replay()
+                e1.record(stream)
+                evs.append((e0, e1))
+        return evs
+
+    def mean_ms(evs):
+        return sum(a.elapsed_time(b) for a, b in evs) / len(evs)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    timed(g_step, args.warmup)
+    torch.cuda.synchronize(dev)
+    uuid = str(getattr(torch.cuda.get_device_properties(dev), "uuid", local))
+    gpu_id = uuid if uuid.startswith("GPU-") else (f"GPU-{uuid}" if len(uuid) > 30 else str(local))
+    clocks = ClockSampler(gpu_id)
+    barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    t_wall0 = time.perf_counter()
+    evs = timed(g_step, args.steps)
+    torch.cuda.synchronize(dev)
+    barrier()
+    t_wall1 = time.perf_counter()
+    clk = clocks.stop()
+    step_ms = max_over_ranks(mean_ms(evs))
+
+    # FFN call alone (the dominant kernels): roofline numerator
+    timed(g_ffn, args.warmup)
+    ffn_evs = timed(g_ffn, args.steps)
+    torch.cuda.synchronize(dev)
+    ffn_ms = max_over_ranks(mean_ms(ffn_evs))
+
+    # end to end through the public API: pinned x in, forward, y out, every step
+    x_host = torch.from_numpy(L.x_bf16.view(np.int16).copy()).pin_memory()
+    y_host = torch.empty((T, cfg.H), dtype=torch.float32).pin_memory()
+    e2e_steps = max(1, min(args.steps, 1000))
+    e2e_evs = []
+    with torch.cuda.stream(stream):
+        for i in range(e2e_steps + 5):
+            flush.fill_(1)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            D.x.copy_(x_host, non_blocking=True)
+            D.forward()
+            y_host.copy_(D.y, non_blocking=True)
+            e1.record(stream)
+            if i >= 5:
+                e2e_evs.append((e0, e1))
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(mean_ms(e2e_evs))
+    st = D.status()
+    if st != B.PW_OK:
+        raise RuntimeError(f"device status after timing: {B.pw_status_string(st)}")
+
+    used = np.unique(D.idx.cpu().numpy())
+    b_layer = layer_bytes(cfg.H, cfg.I, cfg.E, L.q, used, T, bool(np.any(L.bias != 0)))
+    b_ffn = ffn_bytes(cfg.H, cfg.I, L.q, used, T)
+    peak, peak_kind = read_peaks()
+    achieved = b_ffn / (ffn_ms * 1e-3) / 1e9
+    traffic = recorded_traffic()
+    value = world * T / (step_ms * 1e-3)
+    out = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": f"{cfg.name}-shaped MoE decode layer, T={T}", "H": cfg.H,
+                   "E": cfg.E, "I": cfg.I, "k": cfg.k, "parent_bits": cfg.n,
+                   "bits": L.q.tolist(), "experts_used": used.tolist(),
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "flushed before every step (memset of 2.5x L2, outside the step events)",
+                   "timing": "CUDA-graph replay per step, CUDA events on the launching stream"},
+        "effective_gbs": b_layer / (step_ms * 1e-3) / 1e9,
+        "hbm_frac": b_layer / (step_ms * 1e-3) / 1e9 / peak,
+        "bytes_per_step": b_layer,
+        "ffn_ms": ffn_ms,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "kernel": "pw_moe_anyprec_forward (grouping + gate_up + down + combine)",
+                     "peak_kind": f"{peak_kind} copy bandwidth (burst)"},
+        "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(T * cfg.H * 2), "d2h_bytes_per_step": int(T * cfg.H * 4),
+                "ms_per_step": e2e_ms, "path": "pinned x -> pw_route_topk -> "
+                "pw_moe_anyprec_forward -> pinned y, direct calls (no graph)"},
+        "gpu_launches": launches_step * args.steps,
+        "clocks": clk,
+        "wall_s_timed_region": t_wall1 - t_wall0,
+    }
+    if rank == 0 and world == 1:
+        frac = args.cpu_sample_rows or 1.0
+        out["cpu_baseline"] = cpu_baseline(L, T, frac, reps=3)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    del g_step, g_ffn
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_pw(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,238 @@
+/*
+ * pw.h -- C ABI of libpw, a B200 (sm_100a) any-precision MoE decode layer.
+ *
+ * The layer (one MoE layer, decode phase) is:
+ *   router GEMV -> softmax top-k -> substitution (residency rule) or batch remap
+ *   -> fused grouped expert FFN over Any-Precision bit-planes + per-row LUTs
+ *   -> gate-weighted combine.
+ *
+ * Sources, by page and section:
+ *   [PW1]  PagedWeight, "Composants Clés" 1 (Paged Weight Representation): per-(layer, expert,
+ *          module) linear blocks, stacked bit-plane weights with look-up tables, and a Weight
+ *          Page Table holding the desired bitwidth d_i, the committed bitwidth q_i and the page
+ *          state (GPU-resident, CPU-resident, in transfer) of each block.
+ *   [PW3]  PagedWeight, "Composants Clés" 3: one fused mixed-precision kernel reads the
+ *          bit-planes and LUTs directly, each block at its own bitwidth; bitwidth commits only
+ *          happen at safe boundaries.
+ *   [SUB]  "Which Expert Misses Are Worth Waiting For?", "Méthodologie": fetch-every-miss,
+ *          the 0.15 rule, the first-choice rule and the substituted gate mass m.
+ *   [LX1]  LYNX, 1 "Énoncé du Problème": each token independently picks its top-k experts.
+ *   [LX2]  LYNX, 2.1 and 2.2: rank-0 dominates; batch-wide expert scores pick a critical set;
+ *          low-affinity assignments are remapped to it and every token keeps exactly k experts.
+ *
+ * Conventions for every function below:
+ *   - Pointers named *_dev, and every array argument of a compute call, are DEVICE pointers.
+ *     The caller owns and allocates every buffer (inputs, outputs, workspace, page table,
+ *     planes, LUTs).  libpw allocates no device or host memory and keeps no state besides one
+ *     device status word per GPU.
+ *   - Every compute call is asynchronous on `stream` (0 = legacy default stream) and may be
+ *     captured in a CUDA graph.  Argument and shape errors return immediately with
+ *     PW_ERR_INVALID_ARG (or PW_ERR_UNSUPPORTED) and launch nothing.
+ *   - Errors found on the device (a block that is not GPU-resident, a committed bitwidth out
+ *     of range, an expert id out of range, a bounded wait that ran out) never trap: the first
+ *     one is recorded in the device status word and the affected work is skipped (its outputs
+ *     are written as zeros).  pw_get_status() reads and clears it.
+ *   - Floating-point data: bf16 and fp16 are passed as uint16_t bit patterns.
+ */
+#ifndef PW_H_
+#define PW_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st* pw_stream_t; /* same object as cudaStream_t */
+
+typedef enum {
+  PW_OK = 0,
+  PW_ERR_INVALID_ARG = 1,  /* bad pointer, size, shape or config; nothing launched       */
+  PW_ERR_UNSUPPORTED = 2,  /* valid request outside what this build implements          */
+  PW_ERR_CUDA = 3,         /* a CUDA runtime call failed (launch, sync, symbol copy)    */
+  PW_ERR_NOT_RESIDENT = 4, /* device: a used block's page state is not PW_PAGE_GPU      */
+  PW_ERR_TIMEOUT = 5,      /* device: a bounded wait gave up                            */
+  PW_ERR_BAD_EXPERT = 6,   /* device: an expert id outside [0, E)                        */
+  PW_ERR_BAD_BITS = 7      /* device: committed bitwidth outside [min_bits, parent_bits]
+                              or its LUT missing                                        */
+} pw_status;
+
+enum { PW_MOD_GATE_UP = 0, PW_MOD_DOWN = 1 };
+
+/* Page states of a Weight Page Table entry [PW1]. */
+enum { PW_PAGE_GPU = 0, PW_PAGE_CPU = 1, PW_PAGE_XFER = 2 };
+
+/* Assignment rewrite policies [SUB], [LX2]. */
+enum {
+  PW_POLICY_FETCH_ALL = 0,    /* every missing expert is fetched (the rule is the identity)  */
+  PW_POLICY_THRESHOLD = 1,    /* fetch if first choice or gate >= threshold, else substitute */
+  PW_POLICY_FIRST_CHOICE = 2  /* fetch only a missing first choice, substitute the rest      */
+};
+
+/* Substitution actions, one per (token, slot). */
+enum { PW_ACT_HIT = 0, PW_ACT_FETCH = 1, PW_ACT_SUBST = 2 };
+
+#define PW_MIN_BITS 3
+#define PW_MAX_BITS 8
+#define PW_MAX_EXPERTS 1024
+#define PW_MAX_TOPK 16
+#define PW_MAX_TOKENS 4096
+
+/*
+ * One Weight Page Table entry: one linear block (layer, expert, module) [PW1].
+ *   gate_up: rows = 2I, cols = H (rows 0..I-1 gate, rows I..2I-1 up); down: rows = H, cols = I.
+ *   rows % 32 == 0, cols % 128 == 0.
+ *   planes: uint32 [parent_bits][rows][cols/32]; plane p holds bit (parent_bits-1-p) of every
+ *           parent index (plane 0 = most significant); column 32w+j sits at bit j of word w.
+ *           Reading the top q planes gives the q-bit index = top q bits of the parent index.
+ *   lut[b]: fp16 [rows][1<<b] for every b in [min_bits, parent_bits] (NULL otherwise);
+ *           weight(r, c) at bitwidth q = lut[q][r][top q bits of idx(r, c)].
+ *   committed_bits (q_i) is read once per forward call; desired_bits (d_i) is stored for a
+ *   planner and ignored by the kernels.
+ *   tma_desc: filled by pw_block_prepare() (a TMA tensor-map descriptor over `planes`); the
+ *   entry must sit at a 64-byte aligned address on the device.
+ * sizeof(pw_block) == 256.
+ */
+typedef struct pw_block {
+  uint32_t rows;
+  uint32_t cols;
+  uint8_t parent_bits;
+  uint8_t min_bits;
+  uint8_t desired_bits;
+  uint8_t committed_bits;
+  uint8_t state;
+  uint8_t reserved0[3];
+  const uint32_t* planes;
+  const uint16_t* lut[9];
+  uint8_t reserved1[32];
+  uint8_t tma_desc[128];
+} pw_block;
+
+/* The Weight Page Table: device-resident; blocks[(layer * num_experts + e) * 2 + module]. */
+typedef struct pw_page_table {
+  uint32_t num_layers;
+  uint32_t num_experts;
+  pw_block* blocks; /* device pointer, 64-byte aligned */
+} pw_page_table;
+
+/* Routing configuration. */
+typedef struct pw_route_cfg {
+  int32_t k;          /* experts per token, 1..min(E, PW_MAX_TOPK)                      */
+  int32_t renorm;     /* 1: gates = p_sel / sum(p_sel); 0: gates = p_sel                */
+  int32_t policy;     /* PW_POLICY_* (pw_substitute only)                                */
+  float threshold;    /* gate threshold of PW_POLICY_THRESHOLD (0.15 in [SUB])           */
+  int32_t critical_n; /* target size of the critical set (pw_remap; 32 for the LYNX case) */
+} pw_route_cfg;
+
+/* ---------------------------------------------------------------------------------------
+ * pw_block_prepare (host only, no GPU work): validates a host copy of a block entry and
+ * encodes its TMA descriptor.  Call after setting rows/cols/parent_bits/min_bits/planes/lut
+ * and before copying the entry to the device.  Returns PW_ERR_INVALID_ARG for a bad shape,
+ * bitwidth range, missing LUT or misaligned pointer, PW_ERR_CUDA if the driver's
+ * tensor-map encoder is unavailable.
+ * ------------------------------------------------------------------------------------- */
+pw_status pw_block_prepare(pw_block* blk_host);
+
+/* ---------------------------------------------------------------------------------------
+ * pw_pack_bitplanes [PW1]: uint8 parent indices idx[rows][cols] (values < 2^n) into n
+ * bit-planes planes[n][rows][cols/32] in the layout of pw_block.  cols % 32 == 0,
+ * 1 <= n <= 8.  Bits of idx above n are ignored.  Offline (untimed) step.
+ * ------------------------------------------------------------------------------------- */
+pw_status pw_pack_bitplanes(const uint8_t* idx, int rows, int cols, int n, uint32_t* planes,
+                            pw_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * pw_route_topk [LX1]: logits = x W_r^T + bias, then per token the k largest logits in
+ * descending order (equal logits: lower expert index first), and their softmax gates over
+ * all E experts (renormalised over the k when cfg->renorm).
+ *   x_bf16 [T][H] bf16, Wr [E][H] fp32, bias [E] fp32 or NULL.
+ *   logits [T][E] fp32: the float64 dot product plus bias, rounded once to fp32.
+ *   idx [T][k] int32, gate [T][k] fp32 (computed in float64 from the fp32 logits, rounded
+ *   once).  1 <= T <= PW_MAX_TOKENS, 1 <= E <= PW_MAX_EXPERTS, H >= 1.
+ * ------------------------------------------------------------------------------------- */
+pw_status pw_route_topk(const uint16_t* x_bf16, const float* Wr, const float* bias, int T,
+                        int H, int E, const pw_route_cfg* cfg, float* logits, int32_t* idx,
+                        float* gate, pw_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * pw_substitute [SUB]: residency-aware rewrite of the routed assignments, in place.
+ * For each token, slots in rank order: a resident expert is a hit; a missing one is fetched
+ * (kept, counted) when the policy says so (rank 0, or gate >= threshold for
+ * PW_POLICY_THRESHOLD; always for PW_POLICY_FETCH_ALL); otherwise it is replaced by the
+ * highest-logit resident expert not in the token's current set (ties: lower index), keeping
+ * its gate.  With no resident candidate left the miss is fetched.
+ *   logits [T][E] fp32, idx [T][k] int32 (in/out), gate [T][k] fp32, resident [E] uint8.
+ *   action [T][k] uint8 (PW_ACT_*), mass [T] fp32 = substituted gates / all gates of the
+ *   token (float64 sums, rounded once).  action and mass may be NULL.
+ * ------------------------------------------------------------------------------------- */
+pw_status pw_substitute(const float* logits, int32_t* idx, const float* gate,
+                        const uint8_t* resident, int T, int E, const pw_route_cfg* cfg,
+                        uint8_t* action, float* mass, pw_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * pw_remap [LX2]: batch-aware remap to a critical expert set, in place.
+ * S_e = sum of the gates routed to e (float64, ascending (token, slot) order).  The critical
+ * set C is every rank-0 expert plus experts outside it by S_e descending (ties: lower index)
+ * until |C| = cfg->critical_n.  Each slot of rank > 0 whose expert is not in C is replaced,
+ * in rank order, by the highest-logit expert of C not in the token's current set (ties: lower
+ * index), keeping its gate; with none left the slot is kept.  Every token keeps exactly k
+ * distinct experts.
+ *   logits [T][E] fp32, idx [T][k] int32 (in/out), gate [T][k] fp32, critical [E] uint8
+ *   (may be NULL).  Runs as one thread block: T * k <= 8192.
+ * ------------------------------------------------------------------------------------- */
+pw_status pw_remap(const float* logits, int32_t* idx, const float* gate, int T, int E,
+                   const pw_route_cfg* cfg, uint8_t* critical, pw_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * pw_moe_workspace_bytes: device workspace needed by pw_moe_anyprec_forward (0 on bad args).
+ * ------------------------------------------------------------------------------------- */
+size_t pw_moe_workspace_bytes(int T, int k, int E, int H, int I);
+
+/* ---------------------------------------------------------------------------------------
+ * pw_moe_anyprec_forward [PW1][PW3]: grouped expert FFN of one layer, each (expert, module)
+ * block read at its committed bitwidth q straight from its top-q bit-planes and its q-bit
+ * LUT, then the gate-weighted combine.
+ *   for each token t and slot s, e = idx[t][s]:
+ *     g = W_gate(e) x_t, u = W_up(e) x_t, h = SiLU(g) * u, o = W_down(e) h
+ *   y[t] = sum over s (in slot order) of gate[t][s] * o      (fp32 accumulation)
+ *   pt_dev: device page table; layer < num_layers; E must equal its num_experts (checked on
+ *   the device: a mismatch records PW_ERR_INVALID_ARG and the call produces zeros).
+ *   x_bf16 [T][H] bf16, idx [T][k] int32 in [0, E), gate [T][k] fp32, y [T][H] fp32.
+ *   workspace: >= pw_moe_workspace_bytes(T, k, E, H, I) bytes, 256-byte aligned; its
+ *   contents need no initialisation and are overwritten.
+ *   Blocks must be GPU-resident (else PW_ERR_NOT_RESIDENT on the device, that expert's
+ *   contribution is zero).  H % 128 == 0, I % 128 == 0.
+ * ------------------------------------------------------------------------------------- */
+pw_status pw_moe_anyprec_forward(const pw_page_table* pt_dev, int layer, int E,
+                                 const uint16_t* x_bf16, int T, int H, int I, int k,
+                                 const int32_t* idx, const float* gate, float* y, void* workspace,
+                                 size_t ws_bytes, pw_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * pw_commit_bits [PW1][PW3]: set committed_bits of `count` blocks (device arrays block_ids
+ * [count] int32 and q [count] uint8), stream-ordered, so that a commit takes effect exactly
+ * between two forward calls on the stream (a safe boundary).  A block id out of range or a q
+ * outside [min_bits, parent_bits] (or without a LUT) leaves that block unchanged and records
+ * PW_ERR_BAD_BITS.  num_blocks is the table's entry count (num_layers * num_experts * 2).
+ * ------------------------------------------------------------------------------------- */
+pw_status pw_commit_bits(pw_page_table* pt_dev, int num_blocks, const int32_t* block_ids,
+                         const uint8_t* q, int count, pw_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * pw_get_status: synchronises `stream`, then returns and clears the device status word of
+ * the current device (PW_OK if no device-side error was recorded).  Not capturable.
+ * ------------------------------------------------------------------------------------- */
+pw_status pw_get_status(pw_stream_t stream);
+
+/* Human-readable name of a status code (static string). */
+const char* pw_status_string(pw_status s);
+
+/* Library version string (static). */
+const char* pw_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PW_H_ */

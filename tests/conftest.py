@@ -23,3 +23,29 @@ def load_golden(name):
 @pytest.fixture
 def golden():
     return load_golden
+
+
+def _cuda_available():
+    try:
+        import torch
+        return torch.cuda.is_available()
+    except Exception:
+        return False
+
+
+def pytest_collection_modifyitems(config, items):
+    if _cuda_available():
+        return
+    skip = pytest.mark.skip(reason="no CUDA device in this process")
+    for it in items:
+        if "gpu" in it.keywords:
+            it.add_marker(skip)
+
+
+@pytest.fixture(scope="session")
+def libpw():
+    """The built library (built in-tree if missing or stale)."""
+    from any_precision_expert_pw_b200.csrc import build as build_mod
+    build_mod.build()
+    from any_precision_expert_pw_b200 import binding
+    return binding.lib()

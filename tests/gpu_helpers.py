@@ -1,0 +1,30 @@
+"""Shared helpers of the GPU parity tests (comparison rules and sizes)."""
+import numpy as np
+
+from any_precision_expert_pw_b200.inputs import CONFIGS
+
+FFN_RTOL_RMS = 2e-3        # max |y_gpu - y_ref| <= 2e-3 * rms(y_ref)
+GATE_ATOL = 1e-6           # routing gates (fp32 vs float64, rounded once on both sides)
+
+# scaled-down shapes: several tiles, ragged column tails (H or I not a multiple of 1024)
+SCALED = {
+    "tiny": CONFIGS["tiny"],
+    "qwen15": CONFIGS["qwen15_moe_a2.7b"].scaled(H=640, I=384),
+    "mixtral": CONFIGS["mixtral_8x7b"].scaled(H=1152, I=1408),
+    "qwen3next": CONFIGS["qwen3_next_80b_a3b"].scaled(H=384, I=256),
+    "qwen2": CONFIGS["qwen2_57b_a14b"].scaled(H=896, I=640),
+}
+
+
+def ffn_err(y_gpu, y_ref):
+    y_ref = np.asarray(y_ref, np.float64)
+    rms = float(np.sqrt(np.mean(y_ref ** 2)))
+    err = float(np.max(np.abs(np.asarray(y_gpu, np.float64) - y_ref)))
+    return err, rms
+
+
+def assert_ffn_close(y_gpu, y_ref, what=""):
+    err, rms = ffn_err(y_gpu, y_ref)
+    assert rms > 0, what
+    assert err <= FFN_RTOL_RMS * rms, f"{what}: max err {err:.3e} > {FFN_RTOL_RMS} * rms {rms:.3e}"
+    return err / rms

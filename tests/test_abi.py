@@ -1,0 +1,71 @@
+"""The C ABI on the host: the library loads, exports every function include/pw.h declares, and
+rejects bad arguments before launching anything (no GPU needed for these calls)."""
+import ctypes
+import os
+import re
+
+from any_precision_expert_pw_b200 import binding as B
+from conftest import ROOT
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "pw.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(pw_[a-z_]+)\s*\(", src)))
+
+
+def test_header_and_binding_agree(libpw):
+    declared = _declared()
+    assert declared == sorted(B.EXPORTS)
+    for name in declared:
+        assert hasattr(libpw, name), name
+
+
+def test_status_strings_and_version(libpw):
+    assert B.pw_status_string(B.PW_OK) == "PW_OK"
+    assert B.pw_status_string(B.PW_ERR_BAD_BITS) == "PW_ERR_BAD_BITS"
+    assert "sm_100a" in B.pw_version()
+
+
+def test_struct_layouts():
+    assert ctypes.sizeof(B.pw_block) == 256
+    assert B.pw_block.planes.offset == 16 and B.pw_block.lut.offset == 24
+    assert B.pw_block.tma_desc.offset == 128
+
+
+def test_host_argument_checks(libpw):
+    cfg = B.pw_route_cfg(k=2, renorm=1, policy=1, threshold=0.15, critical_n=32)
+    bad = B.PW_ERR_INVALID_ARG
+    assert B.pw_pack_bitplanes(0, 4, 64, 4, 0) == bad
+    assert B.pw_pack_bitplanes(16, 4, 33, 4, 16) == bad           # ragged columns
+    assert B.pw_pack_bitplanes(16, 4, 64, 9, 16) == bad           # n > 8
+    assert B.pw_route_topk(16, 16, 0, 0, 64, 8, cfg, 16, 16, 16) == bad      # T = 0
+    assert B.pw_route_topk(16, 16, 0, 4, 64, 2000, cfg, 16, 16, 16) == bad   # E too large
+    cfg.k = 9
+    assert B.pw_route_topk(16, 16, 0, 4, 64, 8, cfg, 16, 16, 16) == bad      # k > E
+    cfg.k = 2
+    cfg.policy = 7
+    assert B.pw_substitute(16, 16, 16, 16, 4, 8, cfg, 0, 0) == bad           # unknown policy
+    cfg.policy = 1
+    cfg.critical_n = -1
+    assert B.pw_remap(16, 16, 16, 4, 8, cfg, 0) == bad
+    ws = B.pw_moe_workspace_bytes(4, 2, 8, 256, 512)
+    assert ws > 0 and B.pw_moe_workspace_bytes(0, 2, 8, 256, 512) == 0
+    fwd = B.pw_moe_anyprec_forward
+    assert fwd(256, 0, 8, 256, 4, 256, 512, 2, 256, 256, 256, 256, ws - 1) == bad  # small ws
+    assert fwd(256, 0, 8, 256, 4, 200, 512, 2, 256, 256, 256, 256, ws) == bad      # H % 128
+    assert fwd(256, 0, 8, 256, 4, 256, 512, 2, 256, 256, 256, 258, ws) == bad      # ws align
+    assert B.pw_commit_bits(0, 16, 16, 16, 1) == bad
+
+
+def test_block_prepare_rejects_bad_blocks(libpw):
+    blk = B.pw_block()
+    assert B.pw_block_prepare(blk) == B.PW_ERR_INVALID_ARG                 # no planes
+    blk.planes, blk.rows, blk.cols, blk.parent_bits, blk.min_bits = 4096, 64, 100, 8, 3
+    assert B.pw_block_prepare(blk) == B.PW_ERR_INVALID_ARG                 # cols % 128
+    blk.cols = 128
+    assert B.pw_block_prepare(blk) == B.PW_ERR_INVALID_ARG                 # LUTs missing
+    for b in range(3, 9):
+        blk.lut[b] = 4096 * (b + 1)
+    blk.committed_bits = 2
+    assert B.pw_block_prepare(blk) == B.PW_ERR_INVALID_ARG                 # q below min_bits
