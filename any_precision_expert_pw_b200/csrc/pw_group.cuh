@@ -3,6 +3,7 @@
 // set of experts to load grows with the batch -- LYNX, 1 "Énoncé du Problème").
 #pragma once
 #include "pw_common.cuh"
+#include "pw_ffn.cuh"
 
 namespace pw {
 
@@ -72,8 +73,10 @@ __global__ void __launch_bounds__(kGroupThreads) group_kernel(const int32_t* __r
   }
 }
 
-// X[pos][c] = x[token(pos)][c] as fp32 for c < H and 0 for H <= c < ldx; Hbuf[pos][c] = 0 for
-// I <= c < ldh (the FFN streams whole 1024-column stages, so the padding must read as zero).
+// X[pos][xslot(c)] = x[token(pos)][c] as fp32 for c < H and 0 for H <= c < ldx;
+// Hbuf[pos][c] = 0 for I <= c < ldh.  The FFN streams whole 1024-column stages, so the padding
+// must read as zero, and it reads activations in its decode order (xslot, a permutation inside
+// each 32-column group that keeps padding groups whole).
 __global__ void prep_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm,
                             const int32_t* __restrict__ meta, int k, int H, int ldx,
                             float* __restrict__ X, int I, int ldh, float* __restrict__ Hbuf) {
@@ -82,24 +85,29 @@ __global__ void prep_kernel(const uint16_t* __restrict__ x, const int32_t* __res
   if (pos >= n_valid) return;
   const int t = perm[pos] / k;
   for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < ldx; c += gridDim.x * blockDim.x) {
-    X[static_cast<size_t>(pos) * ldx + c] = (c < H) ? bf16_to_f32(x[static_cast<size_t>(t) * H + c])
-                                                     : 0.0f;
+    X[static_cast<size_t>(pos) * ldx + k4::xslot(c)] =
+        (c < H) ? bf16_to_f32(x[static_cast<size_t>(t) * H + c]) : 0.0f;
   }
   for (int c = I + blockIdx.x * blockDim.x + threadIdx.x; c < ldh; c += gridDim.x * blockDim.x)
     Hbuf[static_cast<size_t>(pos) * ldh + c] = 0.0f;
 }
 
-// y[t][r] = sum over slots (in slot order) of gate[t][s] * O[pos(t, s)][r]  (fp32).
+// y[t][r] = sum over slots (in slot order) of gate[t][s] * o[t, s][r], where o is the sum of
+// the down projection's k-slice partials (in slice order).  fp32.
 __global__ void combine_kernel(const float* __restrict__ O, const int32_t* __restrict__ inv,
                                const float* __restrict__ gate, const int32_t* __restrict__ meta,
-                               int T, int k, int H, float* __restrict__ y) {
+                               int T, int k, int H, int kslices, long long slice,
+                               float* __restrict__ y) {
   const int t = blockIdx.y;
   const bool bad = meta[2] != 0;
   for (int r = blockIdx.x * blockDim.x + threadIdx.x; r < H; r += gridDim.x * blockDim.x) {
     float acc = 0.0f;
     for (int s = 0; s < k; ++s) {
       const int pos = inv[t * k + s];
-      if (pos >= 0 && !bad) acc = fmaf(gate[t * k + s], O[static_cast<size_t>(pos) * H + r], acc);
+      if (pos < 0 || bad) continue;
+      float o = 0.0f;
+      for (int j = 0; j < kslices; ++j) o += O[j * slice + static_cast<size_t>(pos) * H + r];
+      acc = fmaf(gate[t * k + s], o, acc);
     }
     y[static_cast<size_t>(t) * H + r] = acc;
   }

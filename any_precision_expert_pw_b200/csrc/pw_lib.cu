@@ -6,6 +6,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <algorithm>
+#include <cmath>
 #include <mutex>
 
 #include "pw.h"
@@ -54,12 +56,12 @@ pw_status device_info(DeviceInfo** out) {
       return PW_ERR_CUDA;
   }
   if (!d.ffn_attr_set) {
-    if (cudaFuncSetAttribute(pw::k4::ffn_kernel<pw::k4::MODE_GATE_UP>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             pw::k4::kSmemBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(pw::k4::ffn_kernel<pw::k4::MODE_DOWN>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             pw::k4::kSmemBytes) != cudaSuccess)
+    if (cudaFuncSetAttribute(pw::k4::ffn_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             pw::k4::Layout<1>::kSmem) != cudaSuccess ||
+        cudaFuncSetAttribute(pw::k4::ffn_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             pw::k4::Layout<2>::kSmem) != cudaSuccess ||
+        cudaFuncSetAttribute(pw::k4::ffn_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             pw::k4::Layout<4>::kSmem) != cudaSuccess)
       return PW_ERR_CUDA;
     d.ffn_attr_set = true;
   }
@@ -111,13 +113,44 @@ Workspace ws_layout(int T, int k, int E, int H, int I) {
   w.meta = take(16);
   w.X = take(4 * TK * w.ldx);
   w.Hbuf = take(4 * TK * w.ldh);
-  w.O = take(4 * TK * H);
+  w.O = take(4 * TK * H * static_cast<size_t>(pw::k4::kMaxKSlices));
   w.total = o;
   return w;
 }
 
 bool cfg_ok(const pw_route_cfg* cfg, int E) {
   return cfg && cfg->k >= 1 && cfg->k <= PW_MAX_TOPK && cfg->k <= E;
+}
+
+// k-slices for the down projection: fill the GPU in whole waves of work items, with at least
+// two 1024-column stages per slice.
+int choose_kslices(int items, int nst, int sms) {
+  int best = 1;
+  double best_eff = 0.0;
+  const int kmax = std::min(pw::k4::kMaxKSlices, std::max(1, nst / 2));
+  for (int ks = 1; ks <= kmax; ++ks) {
+    const double n = static_cast<double>(items) * ks;
+    const double waves = std::ceil(n / sms);
+    const double eff = n / (waves * sms) - 0.01 * ks;
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = ks;
+    }
+  }
+  return best;
+}
+
+pw_status launch_ffn(const pw::k4::Params& p, int max_active, int ntp, int sms,
+                     cudaStream_t st) {
+  const long long items = static_cast<long long>(max_active) * p.tiles * p.kslices;
+  const int grid = static_cast<int>(items < sms ? items : sms);
+  if (ntp == 1)
+    pw::k4::ffn_kernel<1><<<grid, pw::k4::kThreads, pw::k4::Layout<1>::kSmem, st>>>(p);
+  else if (ntp == 2)
+    pw::k4::ffn_kernel<2><<<grid, pw::k4::kThreads, pw::k4::Layout<2>::kSmem, st>>>(p);
+  else
+    pw::k4::ffn_kernel<4><<<grid, pw::k4::kThreads, pw::k4::Layout<4>::kSmem, st>>>(p);
+  return launch_status();
 }
 
 }  // namespace
@@ -276,39 +309,37 @@ pw_status pw_moe_anyprec_forward(const pw_page_table* pt_dev, int layer, int E,
   p.active = active;
   p.meta = meta;
   // gate_up: h = SiLU(W_gate x) * (W_up x)
+  p.mode = pw::k4::MODE_GATE_UP;
   p.rows = 2 * I;
   p.cols = H;
   p.half = I;
   p.tiles = I / pw::k4::kSegRows;
+  p.kslices = 1;
   p.act = X;
   p.ld_act = w.ldx;
   p.out = Hb;
   p.ld_out = w.ldh;
-  {
-    const long long items = static_cast<long long>(max_active) * p.tiles;
-    const int grid = static_cast<int>(items < di->sms ? items : di->sms);
-    pw::k4::ffn_kernel<pw::k4::MODE_GATE_UP>
-        <<<grid, pw::k4::kThreads, pw::k4::kSmemBytes, st>>>(p);
-    if (launch_status() != PW_OK) return PW_ERR_CUDA;
-  }
-  // down: o = W_down h
+  p.out_slice = 0;
+  const int ntp = T == 1 ? 1 : (T == 2 ? 2 : 4);
+  if (launch_ffn(p, max_active, ntp, di->sms, st) != PW_OK) return PW_ERR_CUDA;
+  // down: o = W_down h, split along k so that the grid fills the GPU
+  p.mode = pw::k4::MODE_DOWN;
   p.rows = H;
   p.cols = I;
   p.half = 0;
   p.tiles = H / pw::k4::kRows;
+  p.kslices = choose_kslices(max_active * p.tiles, (I + pw::k4::kStageCols - 1) / pw::k4::kStageCols,
+                             di->sms);
   p.act = Hb;
   p.ld_act = w.ldh;
   p.out = O;
   p.ld_out = H;
-  {
-    const long long items = static_cast<long long>(max_active) * p.tiles;
-    const int grid = static_cast<int>(items < di->sms ? items : di->sms);
-    pw::k4::ffn_kernel<pw::k4::MODE_DOWN><<<grid, pw::k4::kThreads, pw::k4::kSmemBytes, st>>>(p);
-    if (launch_status() != PW_OK) return PW_ERR_CUDA;
-  }
+  p.out_slice = static_cast<long long>(TK) * H;
+  if (launch_ffn(p, max_active, ntp, di->sms, st) != PW_OK) return PW_ERR_CUDA;
   {
     const dim3 g((H + 255) / 256, T);
-    pw::combine_kernel<<<g, 256, 0, st>>>(O, inv, gate, meta, T, k, H, y);
+    pw::combine_kernel<<<g, 256, 0, st>>>(O, inv, gate, meta, T, k, H, p.kslices,
+                                          static_cast<long long>(TK) * H, y);
   }
   return launch_status();
 }

@@ -43,6 +43,8 @@ def parse_args():
     ap.add_argument("--impl", choices=("pw", "reference"), default="pw")
     ap.add_argument("--workload", default=f"{WORKLOAD[0]}:{WORKLOAD[1]}",
                     help="config name:T (default mixtral_8x7b:1)")
+    ap.add_argument("--skip-cpu-baseline", action="store_true",
+                    help="leave out the CPU oracle timing (profiling runs)")
     ap.add_argument("--cpu-sample-rows", type=float, default=None,
                     help="fraction of FFN rows the CPU oracle sample computes")
     return ap.parse_args()
@@ -385,7 +387,7 @@ def run_pw(args):
         "clocks": clk,
         "wall_s_timed_region": t_wall1 - t_wall0,
     }
-    if rank == 0 and world == 1:
+    if rank == 0 and world == 1 and not args.skip_cpu_baseline:
         frac = args.cpu_sample_rows or 1.0
         out["cpu_baseline"] = cpu_baseline(L, T, frac, reps=3)
     if rank == 0:
