@@ -222,9 +222,23 @@ pw_status pw_route_topk(const uint16_t* x_bf16, const float* Wr, const float* bi
   if (!x_bf16 || !Wr || !logits || !idx || !gate) return PW_ERR_INVALID_ARG;
   if (T < 1 || T > PW_MAX_TOKENS || E < 1 || E > PW_MAX_EXPERTS || H < 1 || !cfg_ok(cfg, E))
     return PW_ERR_INVALID_ARG;
-  const dim3 g1((E + pw::kRouteExpertsPerCta - 1) / pw::kRouteExpertsPerCta,
-                (T + pw::kRouteTokensPerCta - 1) / pw::kRouteTokensPerCta);
-  pw::router_logits_kernel<<<g1, 256, 0, as_cuda(stream)>>>(x_bf16, Wr, bias, T, H, E, logits);
+  DeviceInfo* di = nullptr;
+  if (device_info(&di) != PW_OK) return PW_ERR_CUDA;
+  const int e_tiles = (E + pw::kRouteExpertsPerCta - 1) / pw::kRouteExpertsPerCta;
+  const int t_tiles_target = std::max(1, (2 * di->sms + e_tiles - 1) / e_tiles);
+  int tt = (T + t_tiles_target - 1) / t_tiles_target;
+  tt = tt <= 1 ? 1 : tt <= 2 ? 2 : tt <= 4 ? 4 : tt <= 8 ? 8 : 16;
+  const int vec = (H % 8 == 0) && (reinterpret_cast<uintptr_t>(x_bf16) % 16 == 0) &&
+                  (reinterpret_cast<uintptr_t>(Wr) % 16 == 0);
+  const dim3 g1(e_tiles, (T + tt - 1) / tt);
+  cudaStream_t st = as_cuda(stream);
+  switch (tt) {
+    case 1: pw::router_logits_kernel<1><<<g1, 256, 0, st>>>(x_bf16, Wr, bias, T, H, E, vec, logits); break;
+    case 2: pw::router_logits_kernel<2><<<g1, 256, 0, st>>>(x_bf16, Wr, bias, T, H, E, vec, logits); break;
+    case 4: pw::router_logits_kernel<4><<<g1, 256, 0, st>>>(x_bf16, Wr, bias, T, H, E, vec, logits); break;
+    case 8: pw::router_logits_kernel<8><<<g1, 256, 0, st>>>(x_bf16, Wr, bias, T, H, E, vec, logits); break;
+    default: pw::router_logits_kernel<16><<<g1, 256, 0, st>>>(x_bf16, Wr, bias, T, H, E, vec, logits); break;
+  }
   if (launch_status() != PW_OK) return PW_ERR_CUDA;
   pw::topk_kernel<<<(T + 7) / 8, 256, 0, as_cuda(stream)>>>(logits, T, E, cfg->k, cfg->renorm,
                                                             idx, gate);

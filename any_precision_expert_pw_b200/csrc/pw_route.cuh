@@ -12,28 +12,70 @@
 namespace pw {
 
 constexpr int kRouteExpertsPerCta = 8;   // one warp per expert
-constexpr int kRouteTokensPerCta = 8;
+
+__device__ __forceinline__ double bf16lo(uint32_t v) {
+  return static_cast<double>(__uint_as_float(v << 16));
+}
+__device__ __forceinline__ double bf16hi(uint32_t v) {
+  return static_cast<double>(__uint_as_float(v & 0xffff0000u));
+}
 
 // logits[t][e] = fp32(sum_h x[t][h] * Wr[e][h] + bias[e]) with a float64 accumulator.
+// Warp = expert; CTA = 8 experts x TT tokens; each lane takes 8 consecutive h per 256-wide chunk
+// (16-byte loads when `vec`), so the router weights are read once per token tile.
+template <int TT>
 __global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __restrict__ x,
                                                             const float* __restrict__ Wr,
                                                             const float* __restrict__ bias,
-                                                            int T, int H, int E,
+                                                            int T, int H, int E, int vec,
                                                             float* __restrict__ logits) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int e = blockIdx.x * kRouteExpertsPerCta + warp;
   if (e >= E) return;
+  const int t0 = blockIdx.y * TT;
+  const int nt = min(TT, T - t0);
   const float* w = Wr + static_cast<size_t>(e) * H;
-  const int t0 = blockIdx.y * kRouteTokensPerCta;
-  const int t1 = min(T, t0 + kRouteTokensPerCta);
+  double acc[TT];
+#pragma unroll
+  for (int t = 0; t < TT; ++t) acc[t] = 0.0;
+  int hs = 0;
+  if (vec) {
+    const int hv = (H / 256) * 256;
+#pragma unroll 2
+    for (int h0 = lane * 8; h0 < hv; h0 += 256) {
+      const float4 wa = __ldg(reinterpret_cast<const float4*>(w + h0));
+      const float4 wb = __ldg(reinterpret_cast<const float4*>(w + h0 + 4));
+#pragma unroll
+      for (int t = 0; t < TT; ++t) {
+        if (t < nt) {
+          const uint4 xv =
+              __ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(t0 + t) * H + h0));
+          double a = acc[t];
+          a = fma(bf16lo(xv.x), static_cast<double>(wa.x), a);
+          a = fma(bf16hi(xv.x), static_cast<double>(wa.y), a);
+          a = fma(bf16lo(xv.y), static_cast<double>(wa.z), a);
+          a = fma(bf16hi(xv.y), static_cast<double>(wa.w), a);
+          a = fma(bf16lo(xv.z), static_cast<double>(wb.x), a);
+          a = fma(bf16hi(xv.z), static_cast<double>(wb.y), a);
+          a = fma(bf16lo(xv.w), static_cast<double>(wb.z), a);
+          a = fma(bf16hi(xv.w), static_cast<double>(wb.w), a);
+          acc[t] = a;
+        }
+      }
+    }
+    hs = hv;
+  }
+  for (int h = hs + lane; h < H; h += 32) {
+    const double wv = static_cast<double>(w[h]);
+#pragma unroll
+    for (int t = 0; t < TT; ++t)
+      if (t < nt) acc[t] = fma(static_cast<double>(bf16_to_f32(x[static_cast<size_t>(t0 + t) * H + h])), wv, acc[t]);
+  }
   const double b = bias ? static_cast<double>(bias[e]) : 0.0;
-  for (int t = t0; t < t1; ++t) {
-    const uint16_t* xt = x + static_cast<size_t>(t) * H;
-    double acc = 0.0;
-    for (int h = lane; h < H; h += 32)
-      acc = fma(static_cast<double>(bf16_to_f32(xt[h])), static_cast<double>(w[h]), acc);
-    acc = warp_sum_f64(acc);
-    if (lane == 0) logits[static_cast<size_t>(t) * E + e] = static_cast<float>(acc + b);
+#pragma unroll
+  for (int t = 0; t < TT; ++t) {
+    const double v = warp_sum_f64(acc[t]);
+    if (lane == 0 && t < nt) logits[static_cast<size_t>(t0 + t) * E + e] = static_cast<float>(v + b);
   }
 }
 
