@@ -7,15 +7,18 @@
 // rows [32i, 32i+32), optionally split into k-slices whose partial sums the combine adds.
 //
 // Warp roles (one CTA per SM, persistent over the items):
-//   producer (1 warp)   resolves items from the Weight Page Table into a descriptor ring,
-//                       prefetches each item's fp16 LUT one item ahead (1-D bulk copies, two
-//                       staging buffers) and streams, per 1024-column stage, the top-q
-//                       bit-planes of the 32 rows (2-D TMA, 128-byte swizzle) plus the stage's
-//                       activation chunk through a ring of mbarrier-guarded stages;
-//   LUT (2 warps)       turn each item's staged LUT into its decode table in one of two table
-//                       buffers, then signal it ready; a buffer is rewritten only after every
-//                       decode warp has released it, so decode warps never meet a CTA barrier;
-//   decode (16 warps)   take 64 columns of each stage; each thread owns one row (its lane).
+//   producer (1 warp)   resolves the items from the Weight Page Table and streams, per
+//                       1024-column stage, the top-q bit-planes of the 32 rows (2-D TMA,
+//                       128-byte swizzle) plus the stage's activation chunk through a ring of
+//                       mbarrier-guarded stages;
+//   LUT (4 warps)       resolve the items too, read each item's fp16 LUT rows from global memory
+//                       (one row per lane) and build its decode table in one of two table
+//                       buffers, one item ahead of the decode warps, then signal it ready; a
+//                       buffer is rewritten only after every decode warp has released it, so
+//                       decode warps never meet a CTA barrier;
+//   decode (16 warps)   take 64 columns of each stage; each thread owns one row (its lane);
+//   reducer (1 warp)    adds the sixteen per-warp partial sums of every pass in a fixed order
+//                       and writes the output (SiLU(gate) * up for gate_up).
 // Three decode paths, chosen per block by its committed q:
 //   q >= 5  an 8x8 bit-matrix transpose of the q plane words (per 32 columns) yields one index
 //           byte per weight; the table is fp32, lane-interleaved with a 256-byte entry stride
@@ -28,8 +31,7 @@
 //           with the nibble indices as selectors look up four weights at a time.
 // Packed fp32x2 FMAs accumulate.  The decode emits columns as pairs (8b+i, 8b+4+i);
 // activations are stored so every such pair is adjacent (xslot()), two pairs per 16-byte
-// broadcast load.  The sixteen per-warp partial sums of a row are added in a fixed order by
-// whichever decode warp finishes the pass last.
+// broadcast load.
 #pragma once
 #include "pw_common.cuh"
 
@@ -41,16 +43,16 @@ constexpr int kSegRows = 16;
 constexpr int kStageWords = 32;                          // words per row per plane per stage
 constexpr int kStageCols = kStageWords * 32;             // 1024 columns
 constexpr int kDecodeWarps = 16;
-constexpr int kLutWarps = 2;
+constexpr int kLutWarps = 4;
 constexpr int kWarpWords = kStageWords / kDecodeWarps;   // 2 words = 64 columns per warp
 constexpr int kLutWarp0 = kDecodeWarps;
 constexpr int kProducerWarp = kDecodeWarps + kLutWarps;
-constexpr int kThreads = (kProducerWarp + 1) * 32;
+constexpr int kReducerWarp = kProducerWarp + 1;
+constexpr int kThreads = (kReducerWarp + 1) * 32;
 constexpr int kBoxBytes = kSegRows * kStageWords * 4;    // one 16-row TMA box
 constexpr int kPlaneBytes = kRows * kStageWords * 4;     // one plane of a stage
 constexpr int kStagePlaneBytes = PW_MAX_BITS * kPlaneBytes;
 constexpr int kLutBytes = 256 * 256;                     // 2^8 entries x 256-byte stride
-constexpr int kLutStageBytes = kRows * 256 * 2;          // fp16 staging of one tile's LUT
 constexpr int kMaxKSlices = 8;
 constexpr int kDescRing = 4;
 
@@ -65,23 +67,17 @@ __host__ __device__ __forceinline__ int xslot(int c) {
   return (c & ~31) | ((l & 3) << 3) | (((l >> 3) & 3) << 1) | ((l >> 2) & 1);
 }
 
-// A stage slot holds either one 1024-column stage (all q) or, in the one-token kernel, a
-// double-width 2048-column stage for blocks with q <= 4, laid out as two 1024-column halves
-// (planes of half h at h*q*kPlaneBytes; activations of half h at kStagePlaneBytes + h*4 KB),
-// so that low-bitwidth blocks keep as many bytes in flight as high-bitwidth ones.
 template <int NTP>
 struct Layout {
-  static constexpr int kStages = NTP >= 4 ? 2 : 3;
-  static constexpr bool kWide = NTP == 1;
-  static constexpr int kStageXBytes = (kWide ? 2 : NTP) * kStageCols * 4;
+  static constexpr int kStages = NTP == 1 ? 4 : 3;
+  static constexpr int kStageXBytes = NTP * kStageCols * 4;
   static constexpr int kStageBytes = kStagePlaneBytes + kStageXBytes;
   static constexpr int kOffLut = 0;
   static constexpr int kOffStages = kLutBytes;
-  static constexpr int kOffLutStage = kOffStages + kStages * kStageBytes;
-  static constexpr int kOffRed = kOffLutStage + 2 * kLutStageBytes;
+  static constexpr int kOffRed = kOffStages + kStages * kStageBytes;
   static constexpr int kRedBytes = 2 * kDecodeWarps * NTP * 32 * 4;
   static constexpr int kOffDesc = kOffRed + kRedBytes;
-  static constexpr int kDescBytes = 2 * kDescRing * 48;
+  static constexpr int kDescBytes = kDescRing * 48;
   static constexpr int kOffBar = kOffDesc + kDescBytes;
   static constexpr int kBarBytes = (2 * kStages + 8) * 8 + 32;
   static constexpr int kSmem = kOffBar + kBarBytes;
@@ -114,19 +110,18 @@ struct Params {
 
 // What the producer tells the LUT and decode warps about an item (shared-memory rings).
 struct Desc {
-  int valid, status, q, te, pos0, tile, ks, s0, s1, w, pad1, pad2;
+  int valid, status, q, te, pos0, tile, ks, s0, s1, pad0, pad1, pad2;
 };
 static_assert(sizeof(Desc) == 48, "descriptor size");
 
 struct Item {
   const pw_block* blk;
   const uint16_t* lut;
-  int q, tile, ks, te, pos0, segA, segB, s0, s1, w, status;
+  int q, tile, ks, te, pos0, segA, segB, s0, s1, status;
   bool valid;
 };
 
-// wide: the kernel uses double-width stages for q <= 4.
-__device__ __forceinline__ Item resolve(const Params& p, int item, bool wide) {
+__device__ __forceinline__ Item resolve(const Params& p, int item) {
   Item it;
   const int per_expert = p.tiles * p.kslices;
   const int a = item / per_expert;
@@ -146,9 +141,7 @@ __device__ __forceinline__ Item resolve(const Params& p, int item, bool wide) {
     it.segA = it.tile * kRows;
     it.segB = it.segA + kSegRows;
   }
-  it.w = (wide && it.q <= 4) ? 2 : 1;
-  const int scols = kStageCols * it.w;
-  const int nst = (p.cols + scols - 1) / scols;
+  const int nst = (p.cols + kStageCols - 1) / kStageCols;
   it.s0 = (nst * it.ks) / p.kslices;
   it.s1 = (nst * (it.ks + 1)) / p.kslices;
   const bool bits_ok = it.q >= b->min_bits && it.q <= b->parent_bits && it.q >= PW_MIN_BITS &&
@@ -301,26 +294,23 @@ __device__ __forceinline__ void decode_stage(uint32_t planes_off, uint32_t xs_of
 // The stage loop of one pass over an item, one decode warp.  Every argument is a scalar
 // passed by value so nothing of it lives in local memory.  Returns the warp's partial sums
 // (one per token); the caller advances its stage counter by s1 - s0.
-template <int Q, int NT>
+template <int Q, int NT, int NS>
 __device__ __noinline__ float4 run_stages(uint64_t* full, uint64_t* empty,
-                                          volatile int* abort_flag, int n_stages, int stage_bytes,
+                                          volatile int* abort_flag, int stage_bytes,
                                           int words_total, uint32_t lane_base, uint32_t l0,
                                           uint32_t l1, uint32_t l2, uint32_t l3, int s0, int s1,
-                                          uint32_t g, int w) {
+                                          uint32_t g) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint4 reg_lut = make_uint4(l0, l1, l2, l3);
   float2 acc[NT][2];
 #pragma unroll
   for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = make_float2(0.f, 0.f);
   for (int s = s0; s < s1; ++s, ++g) {
-    const int slot = g % n_stages;
-    wait_bar(&full[slot], (g / n_stages) & 1, abort_flag);
+    const int slot = g % NS;
+    wait_bar(&full[slot], (g / NS) & 1, abort_flag);
     const uint32_t st = kLutBytes + slot * stage_bytes;
-    for (int h = 0; h < w; ++h) {
-      if (((s * w + h) * kStageWords + warp * kWarpWords) < words_total)
-        decode_stage<Q, NT>(st + h * Q * kPlaneBytes, st + kStagePlaneBytes + h * kStageCols * 4,
-                            lane_base, reg_lut, warp, lane, acc);
-    }
+    if ((s * kStageWords + warp * kWarpWords) < words_total)
+      decode_stage<Q, NT>(st, st + kStagePlaneBytes, lane_base, reg_lut, warp, lane, acc);
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[slot]);
   }
@@ -331,8 +321,8 @@ __device__ __noinline__ float4 run_stages(uint64_t* full, uint64_t* empty,
 }
 
 #define PW_RUN_ARGS                                                                          \
-  full, empty, abort_flag, LY::kStages, LY::kStageBytes, words_total, lane_base, reg_lut.x,  \
-      reg_lut.y, reg_lut.z, reg_lut.w, d.s0, d.s1, g, d.w
+  full, empty, abort_flag, LY::kStageBytes, words_total, lane_base, reg_lut.x,               \
+      reg_lut.y, reg_lut.z, reg_lut.w, d.s0, d.s1, g
 
 template <int NT, int NTP>
 __device__ __forceinline__ float4 run_q(const Desc& d, uint64_t* full, uint64_t* empty,
@@ -340,36 +330,62 @@ __device__ __forceinline__ float4 run_q(const Desc& d, uint64_t* full, uint64_t*
                                         uint32_t lane_base, const uint4& reg_lut, uint32_t g) {
   using LY = Layout<NTP>;
   switch (d.q) {
-    case 3: return run_stages<3, NT>(PW_RUN_ARGS);
-    case 4: return run_stages<4, NT>(PW_RUN_ARGS);
-    case 5: return run_stages<5, NT>(PW_RUN_ARGS);
-    case 6: return run_stages<6, NT>(PW_RUN_ARGS);
-    case 7: return run_stages<7, NT>(PW_RUN_ARGS);
-    default: return run_stages<8, NT>(PW_RUN_ARGS);
+    case 3: return run_stages<3, NT, LY::kStages>(PW_RUN_ARGS);
+    case 4: return run_stages<4, NT, LY::kStages>(PW_RUN_ARGS);
+    case 5: return run_stages<5, NT, LY::kStages>(PW_RUN_ARGS);
+    case 6: return run_stages<6, NT, LY::kStages>(PW_RUN_ARGS);
+    case 7: return run_stages<7, NT, LY::kStages>(PW_RUN_ARGS);
+    default: return run_stages<8, NT, LY::kStages>(PW_RUN_ARGS);
   }
 }
 #undef PW_RUN_ARGS
 
-// LUT warp lw (0 or 1), lane = row: staged fp16 [32 rows][2^q] -> decode table in buffer u.
-__device__ __forceinline__ void build_table(const uint16_t* __restrict__ ls, int q, uint32_t u,
-                                            int lw, int lane) {
-  const uint32_t col = u * 128 + lane * 4;
-  if (q >= 5) {  // fp32 entries; rows on lanes, entries on a diagonal (conflict-free reads)
-    const int nv = 1 << q, half = nv >> 1;
-    for (int k = 0; k < half; ++k) {
-      const int v = lw * half + ((lane + k) & (half - 1));
-      *reinterpret_cast<float*>(g_smem + v * 256 + col) = f16_to_f32(ls[(lane << q) + v]);
-    }
-  } else if (q == 4) {  // pair entries a + 16b = (LUT[a], LUT[b]); warp lw takes b in [8lw, 8lw+8)
-    const uint4* row = reinterpret_cast<const uint4*>(ls + (lane << 4));
-    const uint4 v0 = row[0], v1 = row[1];
-    const uint32_t lw8[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    const uint4 hsrc = lw ? v1 : v0;  // entries 8lw .. 8lw+7
-    const uint32_t hw[4] = {hsrc.x, hsrc.y, hsrc.z, hsrc.w};
+// LUT warp lw (0..3), lane = row r of the tile (rows segA.. for lanes 0-15, segB.. for 16-31).
+// fetch_table reads the row's share of its fp16 LUT from global memory into registers; it is
+// issued before the warp waits for a free table buffer, so the load latency overlaps that wait.
+struct LutRegs {
+  uint4 v[8];
+};
+
+__device__ __forceinline__ void fetch_table(const uint16_t* __restrict__ row, int q, int lw,
+                                            LutRegs& r) {
+  if (q >= 5) {  // fp32 table; warp lw takes entries [lw * 2^q/4, (lw+1) * 2^q/4)
+    const int quarter = 1 << (q - 2);
+    const uint4* src = reinterpret_cast<const uint4*>(row + lw * quarter);
 #pragma unroll
-    for (int kb = 0; kb < 8; ++kb) {
-      const uint32_t hi = (kb & 1) ? (hw[kb >> 1] >> 16) : (hw[kb >> 1] & 0xffffu);
-      const int b = lw * 8 + kb;
+    for (int k = 0; k < 8; ++k)
+      if (k < quarter / 8) r.v[k] = __ldg(src + k);
+  } else {  // q <= 4: the whole row (16 or 8 entries)
+    r.v[0] = __ldg(reinterpret_cast<const uint4*>(row));
+    if (q == 4) r.v[1] = __ldg(reinterpret_cast<const uint4*>(row) + 1);
+  }
+}
+
+// The fetched LUT row -> decode table in buffer u (fp32 entries for q >= 5, half2 pair entries
+// for q = 4, low/high byte tables for q = 3).
+__device__ __forceinline__ void store_table(const LutRegs& r, int q, uint32_t u, int lw, int lane) {
+  const uint32_t col = u * 128 + lane * 4;
+  if (q >= 5) {
+    const int quarter = 1 << (q - 2);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (k >= quarter / 8) break;
+      const uint32_t w4[4] = {r.v[k].x, r.v[k].y, r.v[k].z, r.v[k].w};
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const int e = lw * quarter + k * 8 + m;
+        const uint16_t h = static_cast<uint16_t>((m & 1) ? (w4[m >> 1] >> 16) : (w4[m >> 1] & 0xffffu));
+        *reinterpret_cast<float*>(g_smem + e * 256 + col) = f16_to_f32(h);
+      }
+    }
+  } else if (q == 4) {  // pair entries a + 16b = (LUT[a], LUT[b]); warp lw takes b in [4lw, 4lw+4)
+    const uint32_t lw8[8] = {r.v[0].x, r.v[0].y, r.v[0].z, r.v[0].w,
+                             r.v[1].x, r.v[1].y, r.v[1].z, r.v[1].w};
+#pragma unroll
+    for (int kb = 0; kb < 4; ++kb) {
+      const int b = lw * 4 + kb;
+      const uint32_t hw = lw8[b >> 1];
+      const uint32_t hi = (b & 1) ? (hw >> 16) : (hw & 0xffffu);
 #pragma unroll
       for (int a = 0; a < 16; ++a) {
         const uint32_t lo = (a & 1) ? (lw8[a >> 1] >> 16) : (lw8[a >> 1] & 0xffffu);
@@ -377,25 +393,11 @@ __device__ __forceinline__ void build_table(const uint16_t* __restrict__ ls, int
       }
     }
   } else if (lw == 0) {  // q == 3: low-byte / high-byte tables for the register lookup
-    const uint4 row = *reinterpret_cast<const uint4*>(ls + (lane << 3));
-    *reinterpret_cast<uint32_t*>(g_smem + 0 * 256 + col) = __byte_perm(row.x, row.y, 0x6420u);
-    *reinterpret_cast<uint32_t*>(g_smem + 1 * 256 + col) = __byte_perm(row.z, row.w, 0x6420u);
-    *reinterpret_cast<uint32_t*>(g_smem + 2 * 256 + col) = __byte_perm(row.x, row.y, 0x7531u);
-    *reinterpret_cast<uint32_t*>(g_smem + 3 * 256 + col) = __byte_perm(row.z, row.w, 0x7531u);
-  }
-}
-
-// Bounded wait until a shared counter reaches `target` (decode warps, partial-sum buffers).
-__device__ __forceinline__ void wait_count(volatile int* c, int target, volatile int* abort_flag) {
-  if (*c >= target || *abort_flag) return;
-  const unsigned long long t0 = global_ns();
-  while (*c < target) {
-    __nanosleep(64);
-    if (global_ns() - t0 > kWaitLimitNs) {
-      set_status(PW_ERR_TIMEOUT);
-      *abort_flag = 1;
-      return;
-    }
+    const uint4 v = r.v[0];
+    *reinterpret_cast<uint32_t*>(g_smem + 0 * 256 + col) = __byte_perm(v.x, v.y, 0x6420u);
+    *reinterpret_cast<uint32_t*>(g_smem + 1 * 256 + col) = __byte_perm(v.z, v.w, 0x6420u);
+    *reinterpret_cast<uint32_t*>(g_smem + 2 * 256 + col) = __byte_perm(v.x, v.y, 0x7531u);
+    *reinterpret_cast<uint32_t*>(g_smem + 3 * 256 + col) = __byte_perm(v.z, v.w, 0x7531u);
   }
 }
 
@@ -404,20 +406,15 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
   using LY = Layout<NTP>;
   uint8_t* const smem = g_smem;
   uint8_t* stages = smem + LY::kOffStages;
-  uint16_t* lut_stage = reinterpret_cast<uint16_t*>(smem + LY::kOffLutStage);
   float* red = reinterpret_cast<float*>(smem + LY::kOffRed);
-  Desc* pdesc = reinterpret_cast<Desc*>(smem + LY::kOffDesc);
-  Desc* cdesc = pdesc + kDescRing;
+  Desc* cdesc = reinterpret_cast<Desc*>(smem + LY::kOffDesc);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + LY::kOffBar);
   uint64_t* empty = full + LY::kStages;
-  uint64_t* lut_full = empty + LY::kStages;   // [2] staging landed (producer -> LUT warps)
-  uint64_t* lut_empty = lut_full + 2;         // [2] staging consumed (LUT warps -> producer)
-  uint64_t* lut_ready = lut_empty + 2;        // [2] table built (LUT warps -> decode)
+  uint64_t* lut_ready = empty + LY::kStages;  // [2] table built (LUT warps -> decode)
   uint64_t* lut_free = lut_ready + 2;         // [2] table released (decode -> LUT warps)
-  int* counters = reinterpret_cast<int*>(lut_free + 2);
-  int* red_arrived = counters;                // [2] monotonic, per pass parity
-  int* red_done = counters + 2;               // [2] monotonic, per pass parity
-  volatile int* abort_flag = counters + 4;
+  uint64_t* red_full = lut_free + 2;          // [2] partial sums written (decode -> reducer)
+  uint64_t* red_free = red_full + 2;          // [2] partial sums consumed (reducer -> decode)
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(red_free + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (smem_u32(smem) & 1023) {  // the swizzled TMA layout needs 1 KB alignment
@@ -430,12 +427,11 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
       mbar_init(&empty[s], kDecodeWarps);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&lut_full[b], 1);
-      mbar_init(&lut_empty[b], kLutWarps);
       mbar_init(&lut_ready[b], kLutWarps);
       mbar_init(&lut_free[b], kDecodeWarps);
+      mbar_init(&red_full[b], kDecodeWarps);
+      mbar_init(&red_free[b], 1);
     }
-    for (int i = 0; i < 4; ++i) counters[i] = 0;
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -444,80 +440,34 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
   const int n_items = p.meta[0] * p.tiles * p.kslices;
 
   if (warp == kProducerWarp) {
-    // ---------------- producer: one thread resolves items and issues every copy ----------
+    // ---------------- producer: one thread streams every stage ----------------
     if (lane != 0) return;
-    const int nst1k = (p.cols + kStageCols - 1) / kStageCols;
     uint32_t g = 0;
-    auto issue_item = [&](const Item& it, uint32_t j) {
-      const int b = j & 1;
-      wait_bar(&lut_empty[b], ((j >> 1) & 1) ^ 1, abort_flag);
-      Desc& d = pdesc[j % kDescRing];
-      d.valid = it.valid;
-      d.status = it.status;
-      d.q = it.q;
-      d.te = it.te;
-      d.pos0 = it.pos0;
-      d.tile = it.tile;
-      d.ks = it.ks;
-      d.s0 = it.s0;
-      d.s1 = it.s1;
-      d.w = it.w;
-      if (it.valid) {
-        const uint32_t seg_lut = static_cast<uint32_t>(kSegRows) << it.q << 1;  // bytes
-        uint16_t* ls = lut_stage + b * (kLutStageBytes / 2);
-        mbar_arrive_expect_tx(&lut_full[b], 2 * seg_lut);
-        bulk_g2s(ls, it.lut + (static_cast<size_t>(it.segA) << it.q), seg_lut, &lut_full[b]);
-        bulk_g2s(ls + (kSegRows << it.q), it.lut + (static_cast<size_t>(it.segB) << it.q),
-                 seg_lut, &lut_full[b]);
-      } else {
-        mbar_arrive(&lut_full[b]);
-      }
-    };
-    int item = blockIdx.x;
-    uint32_t j = 0;
-    Item cur;
-    if (item < n_items) {
-      cur = resolve(p, item, LY::kWide);
-      issue_item(cur, 0);
-    }
-    for (; item < n_items; item += gridDim.x, ++j) {
-      const int next = item + gridDim.x;
-      Item nxt;
-      if (next < n_items) {  // the next item's LUT lands while this item streams
-        nxt = resolve(p, next, LY::kWide);
-        issue_item(nxt, j + 1);
-      }
-      if (cur.valid) {
-        const void* desc = cur.blk->tma_desc;
-        prefetch_desc(desc);
-        for (int ch = 0; ch < cur.te; ch += NTP) {
-          const int ntok = min(NTP, cur.te - ch);
-          for (int s = cur.s0; s < cur.s1; ++s, ++g) {
-            const int slot = g % LY::kStages;
-            wait_bar(&empty[slot], ((g / LY::kStages) & 1) ^ 1, abort_flag);
-            uint8_t* st = stages + slot * LY::kStageBytes;
-            const int chunks = min(cur.w, nst1k - s * cur.w);  // 1024-column chunks present
-            mbar_arrive_expect_tx(&full[slot],
-                                  chunks * (cur.q * kPlaneBytes + ntok * kStageCols * 4));
-            for (int h = 0; h < chunks; ++h) {
-              const int c1k = s * cur.w + h;
-              uint8_t* sp = st + h * cur.q * kPlaneBytes;
-              for (int pl = 0; pl < cur.q; ++pl) {
-                tma_g2s_2d(sp + pl * kPlaneBytes, desc, c1k * kStageWords, pl * p.rows + cur.segA,
-                           &full[slot]);
-                tma_g2s_2d(sp + pl * kPlaneBytes + kBoxBytes, desc, c1k * kStageWords,
-                           pl * p.rows + cur.segB, &full[slot]);
-              }
-              for (int t = 0; t < ntok; ++t)
-                bulk_g2s(st + kStagePlaneBytes + (h + t) * kStageCols * 4,
-                         p.act + static_cast<size_t>(cur.pos0 + ch + t) * p.ld_act +
-                             static_cast<size_t>(c1k) * kStageCols,
-                         kStageCols * 4, &full[slot]);
-            }
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+      const Item cur = resolve(p, item);
+      if (!cur.valid) continue;
+      const void* desc = cur.blk->tma_desc;
+      prefetch_desc(desc);
+      for (int ch = 0; ch < cur.te; ch += NTP) {
+        const int ntok = min(NTP, cur.te - ch);
+        for (int s = cur.s0; s < cur.s1; ++s, ++g) {
+          const int slot = g % LY::kStages;
+          wait_bar(&empty[slot], ((g / LY::kStages) & 1) ^ 1, abort_flag);
+          uint8_t* st = stages + slot * LY::kStageBytes;
+          mbar_arrive_expect_tx(&full[slot], cur.q * kPlaneBytes + ntok * kStageCols * 4);
+          for (int pl = 0; pl < cur.q; ++pl) {
+            tma_g2s_2d(st + pl * kPlaneBytes, desc, s * kStageWords, pl * p.rows + cur.segA,
+                       &full[slot]);
+            tma_g2s_2d(st + pl * kPlaneBytes + kBoxBytes, desc, s * kStageWords,
+                       pl * p.rows + cur.segB, &full[slot]);
           }
+          for (int t = 0; t < ntok; ++t)
+            bulk_g2s(st + kStagePlaneBytes + t * kStageCols * 4,
+                     p.act + static_cast<size_t>(cur.pos0 + ch + t) * p.ld_act +
+                         static_cast<size_t>(s) * kStageCols,
+                     kStageCols * 4, &full[slot]);
         }
       }
-      cur = nxt;
     }
     // drain: every issued copy has landed before the block exits
     for (uint32_t d = (g > LY::kStages ? g - LY::kStages : 0); d < g; ++d)
@@ -525,22 +475,67 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
     return;
   }
 
+  if (warp == kReducerWarp) {
+    // ---------------- reducer: sixteen partial sums per row, in warp order ----------------
+    uint32_t rc = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+      const Item it = resolve(p, item);
+      if (!it.valid) continue;
+      for (int ch = 0; ch < it.te; ch += NTP, ++rc) {
+        const int ntok = min(NTP, it.te - ch);
+        const int par = rc & 1;
+        wait_bar(&red_full[par], (rc >> 1) & 1, abort_flag);
+        const float* rb = red + par * (kDecodeWarps * NTP * 32);
+        for (int t = 0; t < ntok; ++t) {
+          float tot = 0.f;
+#pragma unroll
+          for (int w = 0; w < kDecodeWarps; ++w) tot += rb[(w * NTP + t) * 32 + lane];
+          const size_t row = static_cast<size_t>(it.pos0 + ch + t) * p.ld_out;
+          if (p.mode == MODE_GATE_UP) {
+            const float up = __shfl_down_sync(0xffffffffu, tot, 16);
+            if (lane < kSegRows) {
+              const float h = tot / (1.0f + expf(-tot)) * up;
+              p.out[row + xslot(it.tile * kSegRows + lane)] = h;
+            }
+          } else {
+            p.out[it.ks * p.out_slice + row + it.tile * kRows + lane] = tot;
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&red_free[par]);
+      }
+    }
+    return;
+  }
+
   if (warp >= kLutWarp0) {
-    // ---------------- LUT warps: staged fp16 LUT -> decode table ----------------
+    // ---------------- LUT warps: item descriptors and decode tables ----------------
     const int lw = warp - kLutWarp0;
     uint32_t j = 0;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++j) {
-      const int b = j & 1;
-      wait_bar(&lut_full[b], (j >> 1) & 1, abort_flag);
-      const Desc d = pdesc[j % kDescRing];
-      wait_bar(&lut_free[b], ((j >> 1) & 1) ^ 1, abort_flag);  // decode warps left item j-2
-      if (d.valid) build_table(lut_stage + b * (kLutStageBytes / 2), d.q, b, lw, lane);
-      if (lw == 0 && lane == 0) cdesc[j % kDescRing] = d;
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&lut_empty[b]);
-        mbar_arrive(&lut_ready[b]);
+      const uint32_t u = j & 1;
+      const Item it = resolve(p, item);
+      LutRegs lr;
+      if (it.valid) {
+        const int r = lane < kSegRows ? it.segA + lane : it.segB + (lane - kSegRows);
+        fetch_table(it.lut + (static_cast<size_t>(r) << it.q), it.q, lw, lr);
       }
+      wait_bar(&lut_free[u], ((j >> 1) & 1) ^ 1, abort_flag);  // decode warps left item j-2
+      if (it.valid) store_table(lr, it.q, u, lw, lane);
+      if (lw == 0 && lane == 0) {
+        Desc& d = cdesc[j % kDescRing];
+        d.valid = it.valid;
+        d.status = it.status;
+        d.q = it.q;
+        d.te = it.te;
+        d.pos0 = it.pos0;
+        d.tile = it.tile;
+        d.ks = it.ks;
+        d.s0 = it.s0;
+        d.s1 = it.s1;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&lut_ready[u]);
     }
     return;
   }
@@ -595,46 +590,15 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&lut_free[u]);
       }
-      // partial sums: buffer rc & 1 is free once pass rc - 2 has been reduced
+      // partial sums into buffer rc & 1 once the reducer has consumed pass rc - 2
       const int par = rc & 1;
-      const int k = static_cast<int>(rc >> 1);
-      if (lane == 0) wait_count(&red_done[par], k, abort_flag);
-      __syncwarp();
+      wait_bar(&red_free[par], ((rc >> 1) & 1) ^ 1, abort_flag);
       float* rb = red + par * (kDecodeWarps * NTP * 32);
       const float part[4] = {pv.x, pv.y, pv.z, pv.w};
 #pragma unroll
       for (int t = 0; t < NTP; ++t) rb[(warp * NTP + t) * 32 + lane] = part[t];
       __syncwarp();
-      int last = 0;
-      if (lane == 0) {
-        __threadfence_block();
-        last = atomicAdd(&red_arrived[par], 1) == kDecodeWarps * (k + 1) - 1;
-      }
-      last = __shfl_sync(0xffffffffu, last, 0);
-      if (last) {  // the last warp to finish adds the sixteen partials in warp order
-        __threadfence_block();
-        for (int t = 0; t < ntok; ++t) {
-          float tot = 0.f;
-#pragma unroll
-          for (int w = 0; w < kDecodeWarps; ++w)
-            tot += *reinterpret_cast<volatile float*>(&rb[(w * NTP + t) * 32 + lane]);
-          const size_t row = static_cast<size_t>(d.pos0 + ch + t) * p.ld_out;
-          if (p.mode == MODE_GATE_UP) {
-            const float up = __shfl_down_sync(0xffffffffu, tot, 16);
-            if (lane < kSegRows) {
-              const float h = tot / (1.0f + expf(-tot)) * up;
-              p.out[row + xslot(d.tile * kSegRows + lane)] = h;
-            }
-          } else {
-            p.out[d.ks * p.out_slice + row + d.tile * kRows + lane] = tot;
-          }
-        }
-        __syncwarp();
-        if (lane == 0) {
-          __threadfence_block();
-          atomicAdd(&red_done[par], 1);
-        }
-      }
+      if (lane == 0) mbar_arrive(&red_full[par]);
     }
   }
 }
