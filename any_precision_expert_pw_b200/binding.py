@@ -35,8 +35,10 @@ PW_MAX_TOKENS = 4096
 
 # every symbol include/pw.h declares
 EXPORTS = ("pw_block_prepare", "pw_pack_bitplanes", "pw_route_topk", "pw_substitute",
-           "pw_remap", "pw_moe_workspace_bytes", "pw_moe_anyprec_forward", "pw_commit_bits",
-           "pw_get_status", "pw_status_string", "pw_version")
+           "pw_remap", "pw_moe_workspace_bytes", "pw_moe_anyprec_forward",
+           "pw_moe_anyprec_forward_static", "pw_commit_bits", "pw_get_status",
+           "pw_status_string", "pw_version")
+PW_STATIC_WORKSPACE_BYTES = 16 << 20
 
 
 class PwError(RuntimeError):
@@ -87,6 +89,7 @@ def lib() -> ctypes.CDLL:
         L.pw_moe_workspace_bytes.argtypes = [I, I, I, I, I]
         L.pw_moe_workspace_bytes.restype = Z
         L.pw_moe_anyprec_forward.argtypes = [P, I, I, P, I, I, I, I, P, P, P, P, Z, S]
+        L.pw_moe_anyprec_forward_static.argtypes = [P, I, I, P, I, I, I, I, P, P, P, S]
         L.pw_commit_bits.argtypes = [P, I, P, P, I, S]
         L.pw_get_status.argtypes = [S]
         L.pw_status_string.argtypes = [I]
@@ -152,6 +155,14 @@ def pw_moe_anyprec_forward(pt_dev, layer, E, x_bf16, T, H, I, k, idx, gate, y, w
                            ws_bytes, stream=0) -> int:
     return lib().pw_moe_anyprec_forward(pt_dev, layer, E, x_bf16, T, H, I, k, idx, gate, y,
                                         workspace, ws_bytes, stream)
+
+
+def pw_moe_anyprec_forward_static(pt_dev, layer, E, x_bf16, T, H, I, k, idx, gate, y,
+                                  stream=0) -> int:
+    """pw_moe_anyprec_forward with libpw's own fixed scratch array instead of a caller
+    workspace, for callers that cannot allocate device memory (see include/pw.h)."""
+    return lib().pw_moe_anyprec_forward_static(pt_dev, layer, E, x_bf16, T, H, I, k, idx, gate,
+                                               y, stream)
 
 
 def pw_commit_bits(pt_dev, num_blocks, block_ids, q, count, stream=0) -> int:

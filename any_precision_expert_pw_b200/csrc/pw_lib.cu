@@ -118,6 +118,13 @@ Workspace ws_layout(int T, int k, int E, int H, int I) {
   return w;
 }
 
+// Scratch of pw_moe_anyprec_forward_static: one fixed array per GPU that loads the library.
+// Host code must not hand this symbol to a kernel: on the host it only names the array.  The
+// device address is looked up once per device (g_static_ws_addr) and passed as a pointer.
+static __device__ __align__(256) uint8_t g_static_ws[PW_STATIC_WORKSPACE_BYTES];
+void* g_static_ws_addr[kMaxDevices] = {};
+std::mutex g_static_ws_mu;
+
 bool cfg_ok(const pw_route_cfg* cfg, int E) {
   return cfg && cfg->k >= 1 && cfg->k <= PW_MAX_TOPK && cfg->k <= E;
 }
@@ -356,6 +363,29 @@ pw_status pw_moe_anyprec_forward(const pw_page_table* pt_dev, int layer, int E,
                                           static_cast<long long>(TK) * H, y);
   }
   return launch_status();
+}
+
+pw_status pw_moe_anyprec_forward_static(const pw_page_table* pt_dev, int layer, int E,
+                                        const uint16_t* x_bf16, int T, int H, int I, int k,
+                                        const int32_t* idx, const float* gate, float* y,
+                                        pw_stream_t stream) {
+  if (T < 1 || k < 1 || E < 1 || H < 1 || I < 1) return PW_ERR_INVALID_ARG;
+  const size_t need = pw_moe_workspace_bytes(T, k, E, H, I);
+  if (need == 0) return PW_ERR_INVALID_ARG;
+  if (need > PW_STATIC_WORKSPACE_BYTES) return PW_ERR_UNSUPPORTED;  // shape too large for it
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PW_ERR_CUDA;
+  void* ws = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_static_ws_mu);
+    ws = g_static_ws_addr[dev];
+    if (!ws) {  // first call on this device: look up the array's device address
+      if (cudaGetSymbolAddress(&ws, g_static_ws) != cudaSuccess || !ws) return PW_ERR_CUDA;
+      g_static_ws_addr[dev] = ws;
+    }
+  }
+  return pw_moe_anyprec_forward(pt_dev, layer, E, x_bf16, T, H, I, k, idx, gate, y, ws, need,
+                                stream);
 }
 
 pw_status pw_commit_bits(pw_page_table* pt_dev, int num_blocks, const int32_t* block_ids,

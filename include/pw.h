@@ -25,9 +25,10 @@
  *     The caller owns and allocates every buffer (inputs, outputs, workspace, page table,
  *     planes, LUTs).  libpw allocates no device or host memory and keeps no state besides one
  *     device status word per GPU.
- *   - Every compute call is asynchronous on `stream` (0 = legacy default stream) and may be
- *     captured in a CUDA graph.  Argument and shape errors return immediately with
- *     PW_ERR_INVALID_ARG (or PW_ERR_UNSUPPORTED) and launch nothing.
+ *   - Every compute call other than pw_moe_anyprec_forward_static is asynchronous on `stream`
+ *     (0 = legacy default stream) and may be captured in a CUDA graph.  Argument and shape
+ *     errors return immediately with PW_ERR_INVALID_ARG (or PW_ERR_UNSUPPORTED) and launch
+ *     nothing.
  *   - Errors found on the device (a block that is not GPU-resident, a committed bitwidth out
  *     of range, an expert id out of range, a bounded wait that ran out) never trap: the first
  *     one is recorded in the device status word and the affected work is skipped (its outputs
@@ -209,6 +210,30 @@ pw_status pw_moe_anyprec_forward(const pw_page_table* pt_dev, int layer, int E,
                                  const uint16_t* x_bf16, int T, int H, int I, int k,
                                  const int32_t* idx, const float* gate, float* y, void* workspace,
                                  size_t ws_bytes, pw_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * pw_moe_anyprec_forward_static: pw_moe_anyprec_forward without a caller-provided workspace.
+ * The pages have no counterpart to this call; it exists for callers that cannot allocate
+ * device memory for scratch -- for instance a host program that only receives device
+ * pointers from a serving engine which owns and budgets every GPU allocation (weights, KV
+ * cache), or a plain C caller with no device allocator of its own.
+ *   Same arguments and results as pw_moe_anyprec_forward, minus workspace and ws_bytes.
+ *   Scratch: one array of PW_STATIC_WORKSPACE_BYTES inside libpw, present on every GPU that
+ *   loads the library until the process exits.  Shapes whose pw_moe_workspace_bytes(T, k, E,
+ *   H, I) exceeds it return PW_ERR_UNSUPPORTED and launch nothing.
+ *   The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ *   with that device current; make that first call before any stream capture.
+ *   Every call on a device shares the one array and it keeps the last call's contents (the
+ *   forward overwrites every scratch word it reads, so nothing needs clearing); calls that
+ *   overlap on the GPU -- different streams, or different host threads -- race on it and
+ *   must be serialised by the caller.  It allocates no memory (no cudaMalloc or cudaFree).
+ * ------------------------------------------------------------------------------------- */
+#define PW_STATIC_WORKSPACE_BYTES (16u << 20)
+
+pw_status pw_moe_anyprec_forward_static(const pw_page_table* pt_dev, int layer, int E,
+                                        const uint16_t* x_bf16, int T, int H, int I, int k,
+                                        const int32_t* idx, const float* gate, float* y,
+                                        pw_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------
  * pw_commit_bits [PW1][PW3]: set committed_bits of `count` blocks (device arrays block_ids
