@@ -24,6 +24,7 @@ PW_ERR_BAD_BITS = 7
 
 PW_MOD_GATE_UP = 0
 PW_MOD_DOWN = 1
+PW_LAYOUT_ROWS, PW_LAYOUT_TILED_GATE_UP, PW_LAYOUT_TILED_DOWN = 0, 1, 2
 PW_PAGE_GPU, PW_PAGE_CPU, PW_PAGE_XFER = 0, 1, 2
 PW_POLICY_FETCH_ALL, PW_POLICY_THRESHOLD, PW_POLICY_FIRST_CHOICE = 0, 1, 2
 PW_ACT_HIT, PW_ACT_FETCH, PW_ACT_SUBST = 0, 1, 2
@@ -51,9 +52,10 @@ class pw_block(ctypes.Structure):
     _fields_ = [("rows", ctypes.c_uint32), ("cols", ctypes.c_uint32),
                 ("parent_bits", ctypes.c_uint8), ("min_bits", ctypes.c_uint8),
                 ("desired_bits", ctypes.c_uint8), ("committed_bits", ctypes.c_uint8),
-                ("state", ctypes.c_uint8), ("reserved0", ctypes.c_uint8 * 3),
+                ("state", ctypes.c_uint8), ("layout", ctypes.c_uint8),
+                ("reserved0", ctypes.c_uint8 * 2),
                 ("planes", ctypes.c_void_p), ("lut", ctypes.c_void_p * 9),
-                ("reserved1", ctypes.c_uint8 * 32), ("tma_desc", ctypes.c_uint8 * 128)]
+                ("reserved1", ctypes.c_uint8 * 160)]
 
 
 class pw_page_table(ctypes.Structure):
@@ -66,7 +68,7 @@ class pw_route_cfg(ctypes.Structure):
                 ("threshold", ctypes.c_float), ("critical_n", ctypes.c_int32)]
 
 
-assert ctypes.sizeof(pw_block) == 256 and pw_block.tma_desc.offset == 128
+assert ctypes.sizeof(pw_block) == 256 and pw_block.layout.offset == 13
 assert ctypes.sizeof(pw_page_table) == 16 and ctypes.sizeof(pw_route_cfg) == 20
 
 _lib = None
@@ -82,7 +84,7 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(LIB_PATH)
         P, I, Z, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
         L.pw_block_prepare.argtypes = [ctypes.POINTER(pw_block)]
-        L.pw_pack_bitplanes.argtypes = [P, I, I, I, P, S]
+        L.pw_pack_bitplanes.argtypes = [P, I, I, I, I, P, S]
         L.pw_route_topk.argtypes = [P, P, P, I, I, I, ctypes.POINTER(pw_route_cfg), P, P, P, S]
         L.pw_substitute.argtypes = [P, P, P, P, I, I, ctypes.POINTER(pw_route_cfg), P, P, S]
         L.pw_remap.argtypes = [P, P, P, I, I, ctypes.POINTER(pw_route_cfg), P, S]
@@ -131,8 +133,8 @@ def pw_block_prepare(blk: pw_block) -> int:
     return lib().pw_block_prepare(ctypes.byref(blk))
 
 
-def pw_pack_bitplanes(idx, rows, cols, n, planes, stream=0) -> int:
-    return lib().pw_pack_bitplanes(idx, rows, cols, n, planes, stream)
+def pw_pack_bitplanes(idx, rows, cols, n, layout, planes, stream=0) -> int:
+    return lib().pw_pack_bitplanes(idx, rows, cols, n, layout, planes, stream)
 
 
 def pw_route_topk(x_bf16, Wr, bias, T, H, E, cfg, logits, idx, gate, stream=0) -> int:

@@ -91,19 +91,17 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
-// 2-D tensor copy global -> shared through a TMA descriptor held in global memory.
-// c0 is the innermost coordinate (elements), c1 the outer one.
-__device__ __forceinline__ void tma_g2s_2d(void* dst, const void* desc, int c0, int c1,
-                                           uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, "
-      "{%2, %3}], [%4];" ::"r"(smem_u32(dst)),
-      "l"(desc), "r"(c0), "r"(c1), "r"(smem_u32(bar))
-      : "memory");
+// L2 prefetch of `bytes` (multiple of 16) at a 16-byte aligned global address.
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
-__device__ __forceinline__ void prefetch_desc(const void* desc) {
-  asm volatile("prefetch.tensormap [%0];" ::"l"(desc) : "memory");
+// Programmatic dependent launch.  griddep_wait: the calling thread waits until the grids this
+// one depends on have completed and their writes are visible (returns at once for a plain
+// launch).  griddep_launch: this CTA allows the next grid in the stream to be scheduled.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // Named barrier over a subset of warps (id 1..15).

@@ -8,9 +8,10 @@
 //
 // Warp roles (one CTA per SM, persistent over the items):
 //   producer (1 warp)   resolves the items from the Weight Page Table and streams, per
-//                       1024-column stage, the top-q bit-planes of the 32 rows (2-D TMA,
-//                       128-byte swizzle) plus the stage's activation chunk through a ring of
-//                       mbarrier-guarded stages;
+//                       1024-column stage, the top-q bit-planes of the 32 rows (one bulk copy:
+//                       in the tiled plane layout they are one contiguous run, already in the
+//                       order the decode warps read) plus the stage's activation chunk through
+//                       a ring of mbarrier-guarded stages;
 //   LUT (4 warps)       resolve the items too, read each item's fp16 LUT rows from global memory
 //                       (one row per lane) and build its decode table in one of two table
 //                       buffers, one item ahead of the decode warps, then signal it ready; a
@@ -49,12 +50,12 @@ constexpr int kLutWarp0 = kDecodeWarps;
 constexpr int kProducerWarp = kDecodeWarps + kLutWarps;
 constexpr int kReducerWarp = kProducerWarp + 1;
 constexpr int kThreads = (kReducerWarp + 1) * 32;
-constexpr int kBoxBytes = kSegRows * kStageWords * 4;    // one 16-row TMA box
-constexpr int kPlaneBytes = kRows * kStageWords * 4;     // one plane of a stage
+constexpr int kPlaneBytes = kRows * kStageWords * 4;     // one plane of a full stage
 constexpr int kStagePlaneBytes = PW_MAX_BITS * kPlaneBytes;
 constexpr int kLutBytes = 256 * 256;                     // 2^8 entries x 256-byte stride
 constexpr int kMaxKSlices = 8;
 constexpr int kDescRing = 4;
+constexpr int kPrefetchItems = 2;  // down: items per CTA prefetched into L2 before h is ready
 
 // The kernel's dynamic shared memory, named directly (not through a pointer) wherever the
 // decode loop indexes it, so every table gather is one load with a constant base folded in.
@@ -81,7 +82,7 @@ struct Layout {
   static constexpr int kOffBar = kOffDesc + kDescBytes;
   static constexpr int kBarBytes = (2 * kStages + 8) * 8 + 32;
   static constexpr int kSmem = kOffBar + kBarBytes;
-  static_assert(kStageBytes % 1024 == 0 && kOffStages % 1024 == 0, "swizzle alignment");
+  static_assert(kStageBytes % 128 == 0 && kOffStages % 128 == 0, "stage alignment");
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
 };
 
@@ -101,8 +102,10 @@ struct Params {
   const int32_t* offsets;
   const int32_t* active;
   const int32_t* meta;
-  const float* act;  // [pos][ld_act] fp32 activations in xslot order, zero beyond cols
+  const float* act;  // [row][ld_act] fp32 activations in xslot order, zero beyond cols
   int ld_act;
+  const int32_t* act_map;  // non-null: grouped position pos reads row act_map[pos] / act_div
+  int act_div;             // (gate_up: the token of the assignment); null: row = pos
   float* out;        // gate_up: h [pos][ld_out] (xslot order); down: [kslice][pos][ld_out]
   int ld_out;
   long long out_slice;  // elements between k-slices of `out`
@@ -117,7 +120,8 @@ static_assert(sizeof(Desc) == 48, "descriptor size");
 struct Item {
   const pw_block* blk;
   const uint16_t* lut;
-  int q, tile, ks, te, pos0, segA, segB, s0, s1, status;
+  const uint32_t* planes;  // the tile's run of stages (tiled layout)
+  int q, n, tile, ks, te, pos0, segA, segB, s0, s1, status;
   bool valid;
 };
 
@@ -146,7 +150,11 @@ __device__ __forceinline__ Item resolve(const Params& p, int item) {
   it.s1 = (nst * (it.ks + 1)) / p.kslices;
   const bool bits_ok = it.q >= b->min_bits && it.q <= b->parent_bits && it.q >= PW_MIN_BITS &&
                        it.q <= PW_MAX_BITS && b->lut[it.q] != nullptr && b->planes != nullptr;
-  const bool shape_ok = static_cast<int>(b->rows) == p.rows && static_cast<int>(b->cols) == p.cols;
+  it.n = b->parent_bits;
+  it.planes = b->planes + static_cast<size_t>(it.tile) * it.n * kRows * (p.cols / 32);
+  const int want_layout = p.mode == MODE_GATE_UP ? PW_LAYOUT_TILED_GATE_UP : PW_LAYOUT_TILED_DOWN;
+  const bool shape_ok = static_cast<int>(b->rows) == p.rows &&
+                        static_cast<int>(b->cols) == p.cols && b->layout == want_layout;
   const bool resident = b->state == PW_PAGE_GPU;
   it.lut = bits_ok ? b->lut[it.q] : nullptr;
   it.valid = bits_ok && shape_ok && resident;
@@ -215,16 +223,17 @@ __device__ __forceinline__ float2 hi2(const float4& v) { return make_float2(v.z,
 // planes_off / xs_off: byte offsets of the stage's planes and activations in g_smem.
 // reg_lut: the q = 3 tables (low bytes of entries 0-3, 4-7, high bytes of 0-3, 4-7).
 template <int Q, int NT>
-__device__ __forceinline__ void decode_stage(uint32_t planes_off, uint32_t xs_off,
-                                             uint32_t lane_base, const uint4& reg_lut, int warp,
-                                             int lane, float2 (&acc)[NT][2]) {
-  // 128-byte swizzle: 16-byte chunk index XOR (row % 8); this warp owns half a chunk
-  const uint32_t off = planes_off + lane * 128 + (((warp >> 1) ^ (lane & 7)) << 4) +
-                       ((warp & 1) << 3);
+__device__ __forceinline__ void decode_stage(uint32_t planes_off, uint32_t pstride,
+                                             uint32_t xs_off, uint32_t lane_base,
+                                             const uint4& reg_lut, int warp, int lane,
+                                             float2 (&acc)[NT][2]) {
+  // tiled layout: a plane of the stage is [word pair][row][2 words]; this warp's pair is 256
+  // contiguous bytes, one 8-byte row per lane (conflict free)
+  const uint32_t off = planes_off + warp * 256 + lane * 8;
   uint2 P[Q];
 #pragma unroll
   for (int p = 0; p < Q; ++p)
-    P[p] = *reinterpret_cast<const uint2*>(g_smem + off + p * kPlaneBytes);
+    P[p] = *reinterpret_cast<const uint2*>(g_smem + off + p * pstride);
   constexpr int x_stride = kStageCols;
 #pragma unroll
   for (int wi = 0; wi < kWarpWords; ++wi) {
@@ -309,8 +318,10 @@ __device__ __noinline__ float4 run_stages(uint64_t* full, uint64_t* empty,
     const int slot = g % NS;
     wait_bar(&full[slot], (g / NS) & 1, abort_flag);
     const uint32_t st = kLutBytes + slot * stage_bytes;
-    if ((s * kStageWords + warp * kWarpWords) < words_total)
-      decode_stage<Q, NT>(st, st + kStagePlaneBytes, lane_base, reg_lut, warp, lane, acc);
+    const int ws = min(kStageWords, words_total - s * kStageWords);
+    if (warp * kWarpWords < ws)
+      decode_stage<Q, NT>(st, ws * kRows * 4, st + kStagePlaneBytes, lane_base, reg_lut, warp,
+                          lane, acc);
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[slot]);
   }
@@ -417,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
   volatile int* abort_flag = reinterpret_cast<volatile int*>(red_free + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (smem_u32(smem) & 1023) {  // the swizzled TMA layout needs 1 KB alignment
+  if (smem_u32(smem) & 127) {  // stage buffers and tables assume 128-byte alignment
     if (threadIdx.x == 0) set_status(PW_ERR_UNSUPPORTED);
     return;
   }
@@ -436,36 +447,55 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
     mbar_fence_init();
   }
   __syncthreads();
+  // gate_up reads the grouping written by the launch before it; down reads only the page table,
+  // the grouping (complete before gate_up started) and weights until its producer needs h.
+  if (p.mode == MODE_GATE_UP) griddep_wait();
+  griddep_launch();
 
   const int n_items = p.meta[0] * p.tiles * p.kslices;
+  const int words_total = p.cols / 32;
 
   if (warp == kProducerWarp) {
     // ---------------- producer: one thread streams every stage ----------------
     if (lane != 0) return;
+    if (p.mode == MODE_DOWN) {
+      // while the gate_up grid finishes: this CTA's first items' planes into L2, then wait for h
+      for (int item = blockIdx.x, n = 0; item < n_items && n < kPrefetchItems;
+           item += gridDim.x, ++n) {
+        const Item cur = resolve(p, item);
+        if (!cur.valid) continue;
+        for (int s = cur.s0; s < cur.s1; ++s) {
+          const int ws = min(kStageWords, words_total - s * kStageWords);
+          prefetch_l2(cur.planes + static_cast<size_t>(s) * cur.n * kRows * kStageWords,
+                      cur.q * ws * kRows * 4);
+        }
+      }
+      griddep_wait();
+    }
     uint32_t g = 0;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
       const Item cur = resolve(p, item);
       if (!cur.valid) continue;
-      const void* desc = cur.blk->tma_desc;
-      prefetch_desc(desc);
       for (int ch = 0; ch < cur.te; ch += NTP) {
         const int ntok = min(NTP, cur.te - ch);
+        const float* arow[NTP];
+        for (int t = 0; t < ntok; ++t) {
+          const int pos = cur.pos0 + ch + t;
+          const int r = p.act_map ? p.act_map[pos] / p.act_div : pos;
+          arow[t] = p.act + static_cast<size_t>(r) * p.ld_act;
+        }
         for (int s = cur.s0; s < cur.s1; ++s, ++g) {
           const int slot = g % LY::kStages;
           wait_bar(&empty[slot], ((g / LY::kStages) & 1) ^ 1, abort_flag);
           uint8_t* st = stages + slot * LY::kStageBytes;
-          mbar_arrive_expect_tx(&full[slot], cur.q * kPlaneBytes + ntok * kStageCols * 4);
-          for (int pl = 0; pl < cur.q; ++pl) {
-            tma_g2s_2d(st + pl * kPlaneBytes, desc, s * kStageWords, pl * p.rows + cur.segA,
-                       &full[slot]);
-            tma_g2s_2d(st + pl * kPlaneBytes + kBoxBytes, desc, s * kStageWords,
-                       pl * p.rows + cur.segB, &full[slot]);
-          }
+          const int ws = min(kStageWords, words_total - s * kStageWords);
+          const uint32_t pbytes = cur.q * ws * kRows * 4;
+          mbar_arrive_expect_tx(&full[slot], pbytes + ntok * kStageCols * 4);
+          bulk_g2s(st, cur.planes + static_cast<size_t>(s) * cur.n * kRows * kStageWords, pbytes,
+                   &full[slot]);
           for (int t = 0; t < ntok; ++t)
             bulk_g2s(st + kStagePlaneBytes + t * kStageCols * 4,
-                     p.act + static_cast<size_t>(cur.pos0 + ch + t) * p.ld_act +
-                         static_cast<size_t>(s) * kStageCols,
-                     kStageCols * 4, &full[slot]);
+                     arow[t] + static_cast<size_t>(s) * kStageCols, kStageCols * 4, &full[slot]);
         }
       }
     }
@@ -543,7 +573,6 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
   // ---------------- decode warps ----------------
   const int tid = threadIdx.x;
   const int ndec = kDecodeWarps * 32;
-  const int words_total = p.cols / 32;
   uint32_t g = 0, j = 0, rc = 0;
   for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++j) {
     const uint32_t u = j & 1;

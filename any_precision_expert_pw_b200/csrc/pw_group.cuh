@@ -1,4 +1,5 @@
-// K2: token -> expert grouping and activation staging for the grouped FFN.
+// K2: token -> expert grouping, table check and activation staging for the grouped FFN, and
+// the final gate-weighted combine.
 // Assignment a = t*k + slot.  Within an expert the assignments are kept in ascending a (the
 // set of experts to load grows with the batch -- LYNX, 1 "Énoncé du Problème").
 #pragma once
@@ -10,17 +11,18 @@ namespace pw {
 constexpr int kGroupThreads = 1024;
 constexpr int kMaxAssign = 8192;  // T * k handled by the single-CTA grouping step
 
-// counts[E], offsets[E+1], perm[T*k] (grouped position -> assignment), inv[T*k] (assignment ->
-// grouped position, -1 for an invalid expert id), active[E] (experts with work, ascending),
-// meta[0] = number of active experts, meta[1] = number of valid assignments.
-__global__ void __launch_bounds__(kGroupThreads) group_kernel(const int32_t* __restrict__ idx,
-                                                              int TK, int E,
-                                                              int32_t* __restrict__ counts,
-                                                              int32_t* __restrict__ offsets,
-                                                              int32_t* __restrict__ perm,
-                                                              int32_t* __restrict__ inv,
-                                                              int32_t* __restrict__ active,
-                                                              int32_t* __restrict__ meta) {
+// Grouping, run by one CTA.  counts[E], offsets[E+1], perm[T*k] (grouped position ->
+// assignment), inv[T*k] (assignment -> grouped position, -1 for an invalid expert id),
+// active[E] (experts with work, ascending), meta[0] = number of active experts (0 when the page
+// table does not match (layer, E)), meta[1] = number of valid assignments, meta[2] = 1 for a
+// mismatched table.
+__device__ __forceinline__ void group_block(const pw_page_table* __restrict__ pt, int layer,
+                                            const int32_t* __restrict__ idx, int TK, int E,
+                                            int32_t* __restrict__ counts,
+                                            int32_t* __restrict__ offsets,
+                                            int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                                            int32_t* __restrict__ active,
+                                            int32_t* __restrict__ meta) {
   __shared__ int cnt[PW_MAX_EXPERTS];
   __shared__ int off[PW_MAX_EXPERTS + 1];
   __shared__ int act_pos[PW_MAX_EXPERTS + 1];
@@ -40,6 +42,10 @@ __global__ void __launch_bounds__(kGroupThreads) group_kernel(const int32_t* __r
   }
   __syncthreads();
   if (tid == 0) {  // E <= 1024: a serial scan is a few hundred cycles
+    const bool bad = pt->blocks == nullptr || static_cast<unsigned>(layer) >= pt->num_layers ||
+                     static_cast<int>(pt->num_experts) != E ||
+                     (reinterpret_cast<uintptr_t>(pt->blocks) & 63) != 0;
+    if (bad) set_status(PW_ERR_INVALID_ARG);
     int o = 0, na = 0;
     for (int e = 0; e < E; ++e) {
       off[e] = o;
@@ -49,8 +55,9 @@ __global__ void __launch_bounds__(kGroupThreads) group_kernel(const int32_t* __r
     }
     off[E] = o;
     act_pos[E] = na;
-    meta[0] = na;
+    meta[0] = bad ? 0 : na;
     meta[1] = o;
+    meta[2] = bad ? 1 : 0;
   }
   __syncthreads();
   for (int e = tid; e < E; e += blockDim.x) {
@@ -73,23 +80,60 @@ __global__ void __launch_bounds__(kGroupThreads) group_kernel(const int32_t* __r
   }
 }
 
-// X[pos][xslot(c)] = x[token(pos)][c] as fp32 for c < H and 0 for H <= c < ldx;
-// Hbuf[pos][c] = 0 for I <= c < ldh.  The FFN streams whole 1024-column stages, so the padding
-// must read as zero, and it reads activations in its decode order (xslot, a permutation inside
-// each 32-column group that keeps padding groups whole).
-__global__ void prep_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm,
-                            const int32_t* __restrict__ meta, int k, int H, int ldx,
-                            float* __restrict__ X, int I, int ldh, float* __restrict__ Hbuf) {
-  const int n_valid = meta[1];
-  const int pos = blockIdx.y;
-  if (pos >= n_valid) return;
-  const int t = perm[pos] / k;
-  for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < ldx; c += gridDim.x * blockDim.x) {
-    X[static_cast<size_t>(pos) * ldx + k4::xslot(c)] =
-        (c < H) ? bf16_to_f32(x[static_cast<size_t>(t) * H + c]) : 0.0f;
+// The one launch before the grouped FFN.  CTA 0 checks the page table and groups the
+// assignments; CTAs 1.. write X[t][xslot(c)] = x[t][c] as fp32 for c < H and 0 for
+// H <= c < ldx (one row per token: the gate_up producer maps a grouped position to its token),
+// and Hbuf[pos][c] = 0 for I <= c < ldh.  The FFN streams whole 1024-column stages, so the
+// padding must read as zero, and it reads activations in its decode order (xslot, a
+// permutation inside each 32-column group that keeps padding groups whole).  `vec`: x is
+// 16-byte aligned (H is a multiple of 128), so a thread converts 8 columns from one load.
+__global__ void __launch_bounds__(kGroupThreads) setup_kernel(
+    const pw_page_table* __restrict__ pt, int layer, const int32_t* __restrict__ idx, int T,
+    int k, int E, const uint16_t* __restrict__ x, int H, int ldx, int vec, float* __restrict__ X,
+    int I, int ldh, float* __restrict__ Hbuf, int32_t* __restrict__ counts,
+    int32_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+    int32_t* __restrict__ active, int32_t* __restrict__ meta) {
+  griddep_launch();
+  if (blockIdx.x == 0) {
+    group_block(pt, layer, idx, T * k, E, counts, offsets, perm, inv, active, meta);
+    return;
   }
-  for (int c = I + blockIdx.x * blockDim.x + threadIdx.x; c < ldh; c += gridDim.x * blockDim.x)
-    Hbuf[static_cast<size_t>(pos) * ldh + c] = 0.0f;
+  const size_t nthr = static_cast<size_t>(gridDim.x - 1) * blockDim.x;
+  const size_t t0 = static_cast<size_t>(blockIdx.x - 1) * blockDim.x + threadIdx.x;
+  const int g8 = ldx / 8;  // 8-column groups per row
+  for (size_t i = t0; i < static_cast<size_t>(T) * g8; i += nthr) {
+    const size_t t = i / g8;
+    const int c = static_cast<int>(i - t * g8) * 8;  // columns c..c+7 share (c >> 3) & 3
+    float v[8];
+    if (c >= H) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = 0.0f;
+    } else if (vec) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(x + t * H + c));
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        v[2 * j] = __uint_as_float(w[j] << 16);
+        v[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = bf16_to_f32(x[t * H + c + j]);
+    }
+    // columns c+j and c+j+4 land in adjacent slots
+    float* row = X + t * ldx;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      *reinterpret_cast<float2*>(row + k4::xslot(c + j)) = make_float2(v[j], v[j + 4]);
+  }
+  const int padh = ldh - I;
+  if (padh > 0) {
+    const size_t TK = static_cast<size_t>(T) * k;
+    for (size_t i = t0; i < TK * padh; i += nthr) {
+      const size_t pos = i / padh;
+      Hbuf[pos * ldh + I + (i - pos * padh)] = 0.0f;
+    }
+  }
 }
 
 // y[t][r] = sum over slots (in slot order) of gate[t][s] * o[t, s][r], where o is the sum of
@@ -98,6 +142,7 @@ __global__ void combine_kernel(const float* __restrict__ O, const int32_t* __res
                                const float* __restrict__ gate, const int32_t* __restrict__ meta,
                                int T, int k, int H, int kslices, long long slice,
                                float* __restrict__ y) {
+  griddep_wait();  // O is written by the down projection launched just before
   const int t = blockIdx.y;
   const bool bad = meta[2] != 0;
   for (int r = blockIdx.x * blockDim.x + threadIdx.x; r < H; r += gridDim.x * blockDim.x) {

@@ -1,6 +1,5 @@
 // libpw: host side of the C ABI declared in include/pw.h.  One translation unit: the step
 // kernels live in the pw_*.cuh headers included below.
-#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -21,8 +20,7 @@
 static_assert(sizeof(pw_block) == 256, "pw_block layout");
 static_assert(offsetof(pw_block, planes) == 16, "pw_block layout");
 static_assert(offsetof(pw_block, lut) == 24, "pw_block layout");
-static_assert(offsetof(pw_block, tma_desc) == 128, "pw_block layout");
-static_assert(sizeof(CUtensorMap) == 128, "tensor map size");
+static_assert(offsetof(pw_block, layout) == 13, "pw_block layout");
 static_assert(sizeof(pw_page_table) == 16, "pw_page_table layout");
 static_assert(sizeof(pw_route_cfg) == 20, "pw_route_cfg layout");
 
@@ -69,25 +67,6 @@ pw_status device_info(DeviceInfo** out) {
   return PW_OK;
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult qr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) ==
-            cudaSuccess &&
-        qr == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  });
-  return fn;
-}
-
 // Workspace layout of pw_moe_anyprec_forward.
 struct Workspace {
   size_t counts, offsets, perm, inv, active, meta, X, Hbuf, O, total;
@@ -111,7 +90,7 @@ Workspace ws_layout(int T, int k, int E, int H, int I) {
   w.inv = take(4 * TK);
   w.active = take(4 * static_cast<size_t>(E));
   w.meta = take(16);
-  w.X = take(4 * TK * w.ldx);
+  w.X = take(4 * static_cast<size_t>(T) * w.ldx);
   w.Hbuf = take(4 * TK * w.ldh);
   w.O = take(4 * TK * H * static_cast<size_t>(pw::k4::kMaxKSlices));
   w.total = o;
@@ -147,17 +126,36 @@ int choose_kslices(int items, int nst, int sms) {
   return best;
 }
 
+// Launch with programmatic dependent launch allowed: the kernel may be scheduled while the one
+// before it in the stream is still running, and orders itself with griddepcontrol.wait.
+template <typename... KArgs, typename... Args>
+pw_status launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                           cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...) == cudaSuccess ? PW_OK : PW_ERR_CUDA;
+}
+
 pw_status launch_ffn(const pw::k4::Params& p, int max_active, int ntp, int sms,
                      cudaStream_t st) {
   const long long items = static_cast<long long>(max_active) * p.tiles * p.kslices;
   const int grid = static_cast<int>(items < sms ? items : sms);
   if (ntp == 1)
-    pw::k4::ffn_kernel<1><<<grid, pw::k4::kThreads, pw::k4::Layout<1>::kSmem, st>>>(p);
-  else if (ntp == 2)
-    pw::k4::ffn_kernel<2><<<grid, pw::k4::kThreads, pw::k4::Layout<2>::kSmem, st>>>(p);
-  else
-    pw::k4::ffn_kernel<4><<<grid, pw::k4::kThreads, pw::k4::Layout<4>::kSmem, st>>>(p);
-  return launch_status();
+    return launch_dependent(pw::k4::ffn_kernel<1>, dim3(grid), dim3(pw::k4::kThreads),
+                            pw::k4::Layout<1>::kSmem, st, p);
+  if (ntp == 2)
+    return launch_dependent(pw::k4::ffn_kernel<2>, dim3(grid), dim3(pw::k4::kThreads),
+                            pw::k4::Layout<2>::kSmem, st, p);
+  return launch_dependent(pw::k4::ffn_kernel<4>, dim3(grid), dim3(pw::k4::kThreads),
+                          pw::k4::Layout<4>::kSmem, st, p);
 }
 
 }  // namespace
@@ -194,32 +192,24 @@ pw_status pw_block_prepare(pw_block* blk) {
       return PW_ERR_INVALID_ARG;
   }
   if (blk->committed_bits < mn || blk->committed_bits > n) return PW_ERR_INVALID_ARG;
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return PW_ERR_CUDA;
-  // planes viewed as a 2-D uint32 tensor [n * rows][cols / 32]; box = 32 words x 16 rows
-  const cuuint64_t dims[2] = {cols / 32u, static_cast<cuuint64_t>(rows) * n};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols / 32u) * 4u};
-  const cuuint32_t box[2] = {pw::k4::kStageWords, pw::k4::kSegRows};
-  const cuuint32_t estr[2] = {1, 1};
-  CUtensorMap map;
-  memset(&map, 0, sizeof(map));
-  const CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2,
-                         const_cast<uint32_t*>(blk->planes), dims, strides, box, estr,
-                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return PW_ERR_CUDA;
-  memcpy(blk->tma_desc, &map, sizeof(map));
+  if (blk->layout != PW_LAYOUT_TILED_GATE_UP && blk->layout != PW_LAYOUT_TILED_DOWN)
+    return PW_ERR_INVALID_ARG;
   return PW_OK;
 }
 
-pw_status pw_pack_bitplanes(const uint8_t* idx, int rows, int cols, int n, uint32_t* planes,
-                            pw_stream_t stream) {
+pw_status pw_pack_bitplanes(const uint8_t* idx, int rows, int cols, int n, int layout,
+                            uint32_t* planes, pw_stream_t stream) {
   if (!idx || !planes || rows <= 0 || cols <= 0 || cols % 32 || n < 1 || n > 8)
     return PW_ERR_INVALID_ARG;
+  if (layout != PW_LAYOUT_ROWS && layout != PW_LAYOUT_TILED_GATE_UP &&
+      layout != PW_LAYOUT_TILED_DOWN)
+    return PW_ERR_INVALID_ARG;
+  if (layout != PW_LAYOUT_ROWS && (rows % 32 || cols % 128)) return PW_ERR_INVALID_ARG;
   const long long words = static_cast<long long>(rows) * (cols / 32);
   const long long blocks = (words + 7) / 8;
   const int grid = static_cast<int>(blocks < 65535LL * 16 ? blocks : 65535LL * 16);
-  pw::pack_bitplanes_kernel<<<grid, 256, 0, as_cuda(stream)>>>(idx, rows, cols, n, planes);
+  pw::pack_bitplanes_kernel<<<grid, 256, 0, as_cuda(stream)>>>(idx, rows, cols, n, layout,
+                                                                planes);
   return launch_status();
 }
 
@@ -234,21 +224,20 @@ pw_status pw_route_topk(const uint16_t* x_bf16, const float* Wr, const float* bi
   const int e_tiles = (E + pw::kRouteExpertsPerCta - 1) / pw::kRouteExpertsPerCta;
   const int t_tiles_target = std::max(1, (2 * di->sms + e_tiles - 1) / e_tiles);
   int tt = (T + t_tiles_target - 1) / t_tiles_target;
-  tt = tt <= 1 ? 1 : tt <= 2 ? 2 : tt <= 4 ? 4 : tt <= 8 ? 8 : 16;
+  tt = tt <= 1 ? 1 : tt <= 2 ? 2 : 4;
   const int vec = (H % 8 == 0) && (reinterpret_cast<uintptr_t>(x_bf16) % 16 == 0) &&
                   (reinterpret_cast<uintptr_t>(Wr) % 16 == 0);
   const dim3 g1(e_tiles, (T + tt - 1) / tt);
+  const int fuse_k = (e_tiles == 1) ? cfg->k : 0;  // the whole E in one CTA: top-k fused
   cudaStream_t st = as_cuda(stream);
   switch (tt) {
-    case 1: pw::router_logits_kernel<1><<<g1, 256, 0, st>>>(x_bf16, Wr, bias, T, H, E, vec, logits); break;
-    case 2: pw::router_logits_kernel<2><<<g1, 256, 0, st>>>(x_bf16, Wr, bias, T, H, E, vec, logits); break;
-    case 4: pw::router_logits_kernel<4><<<g1, 256, 0, st>>>(x_bf16, Wr, bias, T, H, E, vec, logits); break;
-    case 8: pw::router_logits_kernel<8><<<g1, 256, 0, st>>>(x_bf16, Wr, bias, T, H, E, vec, logits); break;
-    default: pw::router_logits_kernel<16><<<g1, 256, 0, st>>>(x_bf16, Wr, bias, T, H, E, vec, logits); break;
+    case 1: pw::router_logits_kernel<1><<<g1, pw::kRouteThreads, 0, st>>>(x_bf16, Wr, bias, T, H, E, vec, logits, fuse_k, cfg->renorm, idx, gate); break;
+    case 2: pw::router_logits_kernel<2><<<g1, pw::kRouteThreads, 0, st>>>(x_bf16, Wr, bias, T, H, E, vec, logits, fuse_k, cfg->renorm, idx, gate); break;
+    default: pw::router_logits_kernel<4><<<g1, pw::kRouteThreads, 0, st>>>(x_bf16, Wr, bias, T, H, E, vec, logits, fuse_k, cfg->renorm, idx, gate); break;
   }
   if (launch_status() != PW_OK) return PW_ERR_CUDA;
-  pw::topk_kernel<<<(T + 7) / 8, 256, 0, as_cuda(stream)>>>(logits, T, E, cfg->k, cfg->renorm,
-                                                            idx, gate);
+  if (fuse_k) return PW_OK;
+  pw::topk_kernel<<<(T + 7) / 8, 256, 0, st>>>(logits, T, E, cfg->k, cfg->renorm, idx, gate);
   return launch_status();
 }
 
@@ -310,14 +299,16 @@ pw_status pw_moe_anyprec_forward(const pw_page_table* pt_dev, int layer, int E,
   float* O = reinterpret_cast<float*>(base + w.O);
   const int TK = T * k;
 
-  pw::group_kernel<<<1, pw::kGroupThreads, 0, st>>>(idx, TK, E, counts, offsets, perm, inv,
-                                                     active, meta);
-  if (launch_status() != PW_OK) return PW_ERR_CUDA;
-  pw::check_table_kernel<<<1, 32, 0, st>>>(pt_dev, layer, E, meta);
-  if (launch_status() != PW_OK) return PW_ERR_CUDA;
   {
-    const dim3 g((w.ldx + 255) / 256, TK);
-    pw::prep_kernel<<<g, 256, 0, st>>>(x_bf16, perm, meta, k, H, w.ldx, X, I, w.ldh, Hb);
+    // CTA 0 groups; the others convert x (8 columns per thread)
+    const long long groups = static_cast<long long>(T) * (w.ldx / 8) +
+                             static_cast<long long>(TK) * (w.ldh - I) / 8;
+    const long long conv = (groups + pw::kGroupThreads - 1) / pw::kGroupThreads;
+    const int grid = 1 + static_cast<int>(std::min<long long>(std::max(conv, 1LL), 2LL * di->sms));
+    const int vec = (reinterpret_cast<uintptr_t>(x_bf16) % 16) == 0;
+    pw::setup_kernel<<<grid, pw::kGroupThreads, 0, st>>>(pt_dev, layer, idx, T, k, E, x_bf16, H,
+                                                          w.ldx, vec, X, I, w.ldh, Hb, counts,
+                                                          offsets, perm, inv, active, meta);
     if (launch_status() != PW_OK) return PW_ERR_CUDA;
   }
   const int max_active = E < TK ? E : TK;
@@ -338,6 +329,8 @@ pw_status pw_moe_anyprec_forward(const pw_page_table* pt_dev, int layer, int E,
   p.kslices = 1;
   p.act = X;
   p.ld_act = w.ldx;
+  p.act_map = perm;  // grouped position -> assignment t*k+slot -> token row of X
+  p.act_div = k;
   p.out = Hb;
   p.ld_out = w.ldh;
   p.out_slice = 0;
@@ -353,16 +346,19 @@ pw_status pw_moe_anyprec_forward(const pw_page_table* pt_dev, int layer, int E,
                              di->sms);
   p.act = Hb;
   p.ld_act = w.ldh;
+  p.act_map = nullptr;
+  p.act_div = 1;
   p.out = O;
   p.ld_out = H;
   p.out_slice = static_cast<long long>(TK) * H;
   if (launch_ffn(p, max_active, ntp, di->sms, st) != PW_OK) return PW_ERR_CUDA;
   {
     const dim3 g((H + 255) / 256, T);
-    pw::combine_kernel<<<g, 256, 0, st>>>(O, inv, gate, meta, T, k, H, p.kslices,
-                                          static_cast<long long>(TK) * H, y);
+    return launch_dependent(pw::combine_kernel, g, dim3(256), 0, st,
+                            static_cast<const float*>(O), static_cast<const int32_t*>(inv), gate,
+                            static_cast<const int32_t*>(meta), T, k, H, p.kslices,
+                            static_cast<long long>(TK) * H, y);
   }
-  return launch_status();
 }
 
 pw_status pw_moe_anyprec_forward_static(const pw_page_table* pt_dev, int layer, int E,

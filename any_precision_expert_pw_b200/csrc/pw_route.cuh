@@ -11,7 +11,9 @@
 
 namespace pw {
 
-constexpr int kRouteExpertsPerCta = 8;   // one warp per expert
+constexpr int kRouteExpertsPerCta = 8;
+constexpr int kRouteThreads = 256;
+constexpr int kMaxPerLane = PW_MAX_EXPERTS / 32;
 
 __device__ __forceinline__ double bf16lo(uint32_t v) {
   return static_cast<double>(__uint_as_float(v << 16));
@@ -20,75 +22,14 @@ __device__ __forceinline__ double bf16hi(uint32_t v) {
   return static_cast<double>(__uint_as_float(v & 0xffff0000u));
 }
 
-// logits[t][e] = fp32(sum_h x[t][h] * Wr[e][h] + bias[e]) with a float64 accumulator.
-// Warp = expert; CTA = 8 experts x TT tokens; each lane takes 8 consecutive h per 256-wide chunk
-// (16-byte loads when `vec`), so the router weights are read once per token tile.
-template <int TT>
-__global__ void __launch_bounds__(256) router_logits_kernel(const uint16_t* __restrict__ x,
-                                                            const float* __restrict__ Wr,
-                                                            const float* __restrict__ bias,
-                                                            int T, int H, int E, int vec,
-                                                            float* __restrict__ logits) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int e = blockIdx.x * kRouteExpertsPerCta + warp;
-  if (e >= E) return;
-  const int t0 = blockIdx.y * TT;
-  const int nt = min(TT, T - t0);
-  const float* w = Wr + static_cast<size_t>(e) * H;
-  double acc[TT];
-#pragma unroll
-  for (int t = 0; t < TT; ++t) acc[t] = 0.0;
-  int hs = 0;
-  if (vec) {
-    const int hv = (H / 256) * 256;
-#pragma unroll 2
-    for (int h0 = lane * 8; h0 < hv; h0 += 256) {
-      const float4 wa = __ldg(reinterpret_cast<const float4*>(w + h0));
-      const float4 wb = __ldg(reinterpret_cast<const float4*>(w + h0 + 4));
-#pragma unroll
-      for (int t = 0; t < TT; ++t) {
-        if (t < nt) {
-          const uint4 xv =
-              __ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(t0 + t) * H + h0));
-          double a = acc[t];
-          a = fma(bf16lo(xv.x), static_cast<double>(wa.x), a);
-          a = fma(bf16hi(xv.x), static_cast<double>(wa.y), a);
-          a = fma(bf16lo(xv.y), static_cast<double>(wa.z), a);
-          a = fma(bf16hi(xv.y), static_cast<double>(wa.w), a);
-          a = fma(bf16lo(xv.z), static_cast<double>(wb.x), a);
-          a = fma(bf16hi(xv.z), static_cast<double>(wb.y), a);
-          a = fma(bf16lo(xv.w), static_cast<double>(wb.z), a);
-          a = fma(bf16hi(xv.w), static_cast<double>(wb.w), a);
-          acc[t] = a;
-        }
-      }
-    }
-    hs = hv;
-  }
-  for (int h = hs + lane; h < H; h += 32) {
-    const double wv = static_cast<double>(w[h]);
-#pragma unroll
-    for (int t = 0; t < TT; ++t)
-      if (t < nt) acc[t] = fma(static_cast<double>(bf16_to_f32(x[static_cast<size_t>(t0 + t) * H + h])), wv, acc[t]);
-  }
-  const double b = bias ? static_cast<double>(bias[e]) : 0.0;
-#pragma unroll
-  for (int t = 0; t < TT; ++t) {
-    const double v = warp_sum_f64(acc[t]);
-    if (lane == 0 && t < nt) logits[static_cast<size_t>(t0 + t) * E + e] = static_cast<float>(v + b);
-  }
-}
-
-constexpr int kMaxPerLane = PW_MAX_EXPERTS / 32;
-
-// One warp per token: top-k by (logit desc, index asc), softmax over all E in float64.
-__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E,
-                                                   int k, int renorm, int32_t* __restrict__ idx,
-                                                   float* __restrict__ gate) {
+// One warp, one token: top-k by (logit desc, index asc) over l[0..E), softmax over all E in
+// float64, gates rounded once (renormalised over the k when asked).  Every exp is taken once
+// (float64 exp has a long latency): the selected experts' probabilities are read back from the
+// lane that holds them.
+__device__ __forceinline__ void topk_warp(const float* l, int E, int k, int renorm,
+                                          int32_t* __restrict__ idx_out,
+                                          float* __restrict__ gate_out) {
   const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (t >= T) return;
-  const float* l = logits + static_cast<size_t>(t) * E;
   float v[kMaxPerLane];
   float mx = -INFINITY;
 #pragma unroll
@@ -99,62 +40,216 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  double ex[kMaxPerLane];
   double z = 0.0;
 #pragma unroll
-  for (int i = 0; i < kMaxPerLane; ++i)
-    if (lane + 32 * i < E) z += exp(static_cast<double>(v[i]) - static_cast<double>(mx));
+  for (int i = 0; i < kMaxPerLane; ++i) {
+    ex[i] = 0.0;
+    if (lane + 32 * i < E) {
+      ex[i] = exp(static_cast<double>(v[i]) - static_cast<double>(mx));
+      z += ex[i];
+    }
+  }
   z = warp_sum_f64(z);
 
   uint32_t taken = 0;  // bit i: element lane+32i already chosen
-  double psel[PW_MAX_TOPK];
-  int esel[PW_MAX_TOPK];
-  double psum = 0.0;
+  double psum = 0.0, mine = 0.0;
   for (int j = 0; j < k; ++j) {
     float bv = -INFINITY;
     int bi = -1;
+    double be = 0.0;
 #pragma unroll
     for (int i = 0; i < kMaxPerLane; ++i) {
       const int e = lane + 32 * i;
       if (e < E && !((taken >> i) & 1u) && (bi < 0 || v[i] > bv)) {
         bv = v[i];
         bi = e;
+        be = ex[i];
       }
     }
     warp_argmax(bv, bi);
     if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-    const double p = exp(static_cast<double>(bv) - static_cast<double>(mx)) / z;
-    psel[j] = p;
-    esel[j] = bi;
+    // the winner's exp, from the lane whose own candidate it was
+    const double p = __shfl_sync(0xffffffffu, be, bi & 31) / z;
     psum += p;
+    if (lane == j) mine = p;
+    if (lane == 0) idx_out[j] = bi;
   }
-  if (lane == 0) {
-    for (int j = 0; j < k; ++j) {
-      idx[static_cast<size_t>(t) * k + j] = esel[j];
-      gate[static_cast<size_t>(t) * k + j] =
-          static_cast<float>(renorm ? psel[j] / psum : psel[j]);
+  if (lane < k) gate_out[lane] = static_cast<float>(renorm ? mine / psum : mine);
+}
+
+// logits[t][e] = fp32(sum_h x[t][h] * Wr[e][h] + bias[e]) with float64 accumulation.
+// CTA = 8 experts x TT tokens; all 256 threads split H (8 consecutive h per thread per
+// 2048-wide chunk, 16-byte loads when `vec`), so every load of a CTA is in flight at once; the
+// 256 partial sums of each (expert, token) are added in a fixed order.  With fuse_k > 0 (the
+// whole E fits one CTA) the CTA then runs the top-k of its tokens as well.
+template <int TT>
+__global__ void __launch_bounds__(kRouteThreads) router_logits_kernel(
+    const uint16_t* __restrict__ x, const float* __restrict__ Wr, const float* __restrict__ bias,
+    int T, int H, int E, int vec, float* __restrict__ logits, int fuse_k, int renorm,
+    int32_t* __restrict__ idx, float* __restrict__ gate) {
+  __shared__ double part[kRouteThreads / 32][kRouteExpertsPerCta][TT];
+  __shared__ float lsm[TT][kRouteExpertsPerCta];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int e0 = blockIdx.x * kRouteExpertsPerCta;
+  const int ne = min(kRouteExpertsPerCta, E - e0);
+  const int t0 = blockIdx.y * TT;
+  const int nt = min(TT, T - t0);
+  double acc[kRouteExpertsPerCta][TT];
+#pragma unroll
+  for (int e = 0; e < kRouteExpertsPerCta; ++e)
+#pragma unroll
+    for (int t = 0; t < TT; ++t) acc[e][t] = 0.0;
+  // Rows past E (or T) are clamped to the last valid one and their sums discarded, so every
+  // load of an iteration is unconditional and all of them are in flight together.
+  const uint16_t* xr[TT];
+  const float* wr[kRouteExpertsPerCta];
+#pragma unroll
+  for (int t = 0; t < TT; ++t) xr[t] = x + static_cast<size_t>(t0 + min(t, nt - 1)) * H;
+#pragma unroll
+  for (int e = 0; e < kRouteExpertsPerCta; ++e)
+    wr[e] = Wr + static_cast<size_t>(e0 + min(e, ne - 1)) * H;
+  if (vec) {
+    // CH chunks of 2048 columns per round (two for a single token, so that both rounds of a
+    // 4096-wide row are loaded at once); a chunk past H re-reads chunk 0 and is not added
+    constexpr int CH = TT == 1 ? 2 : 1;
+    for (int hb = tid * 8; hb < H; hb += CH * kRouteThreads * 8) {
+      uint4 xv[CH][TT];
+      float4 wa[CH][kRouteExpertsPerCta], wb[CH][kRouteExpertsPerCta];
+      bool live[CH];
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        live[c] = hb + c * kRouteThreads * 8 < H;
+        const int h0 = live[c] ? hb + c * kRouteThreads * 8 : hb;
+#pragma unroll
+        for (int t = 0; t < TT; ++t) xv[c][t] = __ldg(reinterpret_cast<const uint4*>(xr[t] + h0));
+#pragma unroll
+        for (int e = 0; e < kRouteExpertsPerCta; ++e) {
+          wa[c][e] = __ldg(reinterpret_cast<const float4*>(wr[e] + h0));
+          wb[c][e] = __ldg(reinterpret_cast<const float4*>(wr[e] + h0 + 4));
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        if (!live[c]) continue;
+#pragma unroll
+        for (int e = 0; e < kRouteExpertsPerCta; ++e) {
+#pragma unroll
+          for (int t = 0; t < TT; ++t) {
+            const uint4 xq = xv[c][t];
+            const float4 a4 = wa[c][e], b4 = wb[c][e];
+            double a = acc[e][t];
+            a = fma(bf16lo(xq.x), static_cast<double>(a4.x), a);
+            a = fma(bf16hi(xq.x), static_cast<double>(a4.y), a);
+            a = fma(bf16lo(xq.y), static_cast<double>(a4.z), a);
+            a = fma(bf16hi(xq.y), static_cast<double>(a4.w), a);
+            a = fma(bf16lo(xq.z), static_cast<double>(b4.x), a);
+            a = fma(bf16hi(xq.z), static_cast<double>(b4.y), a);
+            a = fma(bf16lo(xq.w), static_cast<double>(b4.z), a);
+            a = fma(bf16hi(xq.w), static_cast<double>(b4.w), a);
+            acc[e][t] = a;
+          }
+        }
+      }
     }
+  } else {
+    for (int h = tid; h < H; h += kRouteThreads) {
+      double xv[TT], wv[kRouteExpertsPerCta];
+#pragma unroll
+      for (int t = 0; t < TT; ++t) xv[t] = static_cast<double>(bf16_to_f32(xr[t][h]));
+#pragma unroll
+      for (int e = 0; e < kRouteExpertsPerCta; ++e) wv[e] = static_cast<double>(wr[e][h]);
+#pragma unroll
+      for (int e = 0; e < kRouteExpertsPerCta; ++e)
+#pragma unroll
+        for (int t = 0; t < TT; ++t) acc[e][t] = fma(xv[t], wv[e], acc[e][t]);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < kRouteExpertsPerCta; ++e)
+#pragma unroll
+    for (int t = 0; t < TT; ++t) {
+      const double v = warp_sum_f64(acc[e][t]);
+      if (lane == 0) part[warp][e][t] = v;
+    }
+  __syncthreads();
+  if (tid < kRouteExpertsPerCta * TT) {
+    const int e = tid / TT, t = tid - e * TT;
+    if (e < ne && t < nt) {
+      double s = 0.0;
+#pragma unroll
+      for (int w = 0; w < kRouteThreads / 32; ++w) s += part[w][e][t];
+      const double b = bias ? static_cast<double>(bias[e0 + e]) : 0.0;
+      const float lv = static_cast<float>(s + b);
+      logits[static_cast<size_t>(t0 + t) * E + e0 + e] = lv;
+      lsm[t][e] = lv;
+    }
+  }
+  if (fuse_k > 0) {
+    __syncthreads();
+    for (int t = warp; t < nt; t += kRouteThreads / 32)
+      topk_warp(lsm[t], E, fuse_k, renorm, idx + static_cast<size_t>(t0 + t) * fuse_k,
+                gate + static_cast<size_t>(t0 + t) * fuse_k);
   }
 }
 
-// Highest-logit expert e with allowed[e] and e not in cur[0..k) (ties: lower index); -1 if none.
-__device__ __forceinline__ int best_candidate(const float* __restrict__ l, const uint8_t* allowed,
-                                              int E, const int* cur, int k) {
+// One warp per token: top-k of a logits row in global memory.
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E,
+                                                   int k, int renorm, int32_t* __restrict__ idx,
+                                                   float* __restrict__ gate) {
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  topk_warp(logits + static_cast<size_t>(t) * E, E, k, renorm, idx + static_cast<size_t>(t) * k,
+            gate + static_cast<size_t>(t) * k);
+}
+
+// A token's logits row held by one warp: element e = lane + 32 i in v[i] (-inf past E).
+struct WarpRow {
+  float v[kMaxPerLane];
+};
+
+__device__ __forceinline__ void load_row(const float* __restrict__ l, int E, WarpRow& r) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int i = 0; i < kMaxPerLane; ++i) {
+    const int e = lane + 32 * i;
+    r.v[i] = (e < E) ? l[e] : -INFINITY;
+  }
+}
+
+// Bit i of the result: expert lane + 32 i is one of cur[0..k).
+__device__ __forceinline__ uint32_t lane_set(const int* cur, int k) {
+  const int lane = threadIdx.x & 31;
+  uint32_t m = 0;
+  for (int j = 0; j < k; ++j)
+    if ((cur[j] & 31) == lane) m |= 1u << (cur[j] >> 5);
+  return m;
+}
+
+// Highest-logit expert e with bit (e >> 5) of this lane's `allowed` set and e not in `chosen`
+// (ties: lower index); -1 if none.
+__device__ __forceinline__ int best_candidate(const WarpRow& r, uint32_t allowed, uint32_t chosen,
+                                              int E) {
   const int lane = threadIdx.x & 31;
   float bv = -INFINITY;
   int bi = -1;
-  for (int e = lane; e < E; e += 32) {
-    if (!allowed[e]) continue;
-    bool in_set = false;
-    for (int j = 0; j < k; ++j) in_set |= (cur[j] == e);
-    if (in_set) continue;
-    const float le = l[e];
-    if (bi < 0 || le > bv) {
-      bv = le;
+#pragma unroll
+  for (int i = 0; i < kMaxPerLane; ++i) {
+    const int e = lane + 32 * i;
+    if (e < E && ((allowed >> i) & 1u) && !((chosen >> i) & 1u) && (bi < 0 || r.v[i] > bv)) {
+      bv = r.v[i];
       bi = e;
     }
   }
   warp_argmax(bv, bi);
   return bi;
+}
+
+// Replace cur[s] by c in the per-lane chosen mask.
+__device__ __forceinline__ void swap_chosen(uint32_t& chosen, int old_e, int new_e) {
+  const int lane = threadIdx.x & 31;
+  if ((old_e & 31) == lane) chosen &= ~(1u << (old_e >> 5));
+  if ((new_e & 31) == lane) chosen |= 1u << (new_e >> 5);
 }
 
 __global__ void __launch_bounds__(256) substitute_kernel(
@@ -174,7 +269,15 @@ __global__ void __launch_bounds__(256) substitute_kernel(
     if (lane == 0) set_status(PW_ERR_BAD_EXPERT);
     return;
   }
-  const float* l = logits + static_cast<size_t>(t) * E;
+  WarpRow row;
+  load_row(logits + static_cast<size_t>(t) * E, E, row);
+  uint32_t res = 0;
+#pragma unroll
+  for (int i = 0; i < kMaxPerLane; ++i) {
+    const int e = lane + 32 * i;
+    if (e < E && resident[e]) res |= 1u << i;
+  }
+  uint32_t chosen = lane_set(cur, k);
   double sub = 0.0, tot = 0.0;
   uint8_t act[PW_MAX_TOPK];
   for (int s = 0; s < k; ++s) {
@@ -190,8 +293,9 @@ __global__ void __launch_bounds__(256) substitute_kernel(
     else fetch = (s == 0) || (g >= threshold);
     act[s] = PW_ACT_FETCH;
     if (!fetch) {
-      const int c = best_candidate(l, resident, E, cur, k);
+      const int c = best_candidate(row, res, chosen, E);
       if (c >= 0) {
+        swap_chosen(chosen, cur[s], c);
         cur[s] = c;
         act[s] = PW_ACT_SUBST;
         sub += static_cast<double>(g);
@@ -263,14 +367,25 @@ __global__ void __launch_bounds__(1024) remap_kernel(const float* __restrict__ l
   if (critical)
     for (int e = tid; e < E; e += blockDim.x) critical[e] = crit[e];
   const int warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
+  uint32_t crit_bits = 0;
+#pragma unroll
+  for (int i = 0; i < kMaxPerLane; ++i) {
+    const int e = lane + 32 * i;
+    if (e < E && crit[e]) crit_bits |= 1u << i;
+  }
   for (int t = warp; t < T; t += nw) {
     int cur[PW_MAX_TOPK];
     for (int j = 0; j < k; ++j) cur[j] = idx[static_cast<size_t>(t) * k + j];
-    const float* l = logits + static_cast<size_t>(t) * E;
+    WarpRow row;
+    load_row(logits + static_cast<size_t>(t) * E, E, row);
+    uint32_t chosen = lane_set(cur, k);
     for (int s = 1; s < k; ++s) {
       if (crit[cur[s]]) continue;
-      const int c = best_candidate(l, crit, E, cur, k);
-      if (c >= 0) cur[s] = c;
+      const int c = best_candidate(row, crit_bits, chosen, E);
+      if (c >= 0) {
+        swap_chosen(chosen, cur[s], c);
+        cur[s] = c;
+      }
     }
     __syncwarp();
     if (lane == 0)

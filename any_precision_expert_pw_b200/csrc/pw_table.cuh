@@ -1,6 +1,5 @@
 // Weight Page Table kernels (PagedWeight, "Composants Clés" 1 and 3): stream-ordered commits of
-// q_i, so a commit lands exactly between two forward calls (a safe boundary), and the per-call
-// check of the table against the caller's layer and expert count.
+// q_i, so a commit lands exactly between two forward calls (a safe boundary).
 #pragma once
 #include "pw_common.cuh"
 
@@ -25,20 +24,6 @@ __global__ void commit_bits_kernel(pw_page_table* __restrict__ pt, int num_block
     return;
   }
   b->committed_bits = static_cast<uint8_t>(qq);
-}
-
-// meta[2] = 1 (and no active experts) when the table does not match (layer, E).
-__global__ void check_table_kernel(const pw_page_table* __restrict__ pt, int layer, int E,
-                                   int32_t* __restrict__ meta) {
-  if (threadIdx.x != 0) return;
-  const bool bad = pt->blocks == nullptr || static_cast<unsigned>(layer) >= pt->num_layers ||
-                   static_cast<int>(pt->num_experts) != E ||
-                   (reinterpret_cast<uintptr_t>(pt->blocks) & 63) != 0;
-  if (bad) {
-    set_status(PW_ERR_INVALID_ARG);
-    meta[0] = 0;
-  }
-  meta[2] = bad ? 1 : 0;
 }
 
 }  // namespace pw

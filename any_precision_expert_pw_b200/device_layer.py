@@ -50,9 +50,10 @@ class DeviceLayer:
         for e in range(cfg.E):
             for m in (MOD_GATE_UP, MOD_DOWN):
                 R, C = L.block_shape(m)
-                planes = torch.empty((n, R, C // 32), dtype=torch.int32, device=self.device)
+                layout = B.PW_LAYOUT_TILED_GATE_UP if m == MOD_GATE_UP else B.PW_LAYOUT_TILED_DOWN
+                planes = torch.empty((n * R * (C // 32),), dtype=torch.int32, device=self.device)
                 idx_d = _dev_tensor(L.idx[e][m], self.device)
-                B.check(B.pw_pack_bitplanes(idx_d.data_ptr(), R, C, n, planes.data_ptr(),
+                B.check(B.pw_pack_bitplanes(idx_d.data_ptr(), R, C, n, layout, planes.data_ptr(),
                                             self.stream), "pw_pack_bitplanes")
                 del idx_d
                 parts = [L.lut[e][m][b].view(np.int16).reshape(-1) for b in range(MIN_BITS, n + 1)]
@@ -63,6 +64,7 @@ class DeviceLayer:
                 q = int(L.q[e, m])
                 blk.desired_bits = blk.committed_bits = q
                 blk.state = B.PW_PAGE_GPU
+                blk.layout = layout
                 blk.planes = planes.data_ptr()
                 off = 0
                 for b in range(MIN_BITS, n + 1):

@@ -66,13 +66,16 @@ def read_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+# the sources of the kernels pw_moe_anyprec_forward launches (and their launch logic)
+FORWARD_SOURCES = ("pw_common.cuh", "pw_ffn.cuh", "pw_group.cuh", "pw_lib.cu")
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "any_precision_expert_pw_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, f), "rb") as fh:
-                h.update(fh.read())
+    for f in FORWARD_SOURCES:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
     return h.hexdigest()[:16]
 
 
@@ -276,7 +279,9 @@ def run_pw(args):
     g_ffn = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_ffn, stream=stream):
         D.ffn()
-    launches_step = 2 + (0 if cfg.policy == POLICY_NONE else 1) + 6
+    # router (+ top-k, fused into it when the E experts fit one CTA of 8), the assignment
+    # rewrite if any, then setup, gate_up, down and combine
+    launches_step = (1 if cfg.E <= 8 else 2) + (0 if cfg.policy == POLICY_NONE else 1) + 4
 
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(int(2.5 * l2), dtype=torch.uint8, device=dev)

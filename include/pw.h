@@ -62,6 +62,13 @@ typedef enum {
 
 enum { PW_MOD_GATE_UP = 0, PW_MOD_DOWN = 1 };
 
+/* Bit-plane layouts written by pw_pack_bitplanes (see pw_block for their definitions). */
+enum {
+  PW_LAYOUT_ROWS = 0,          /* [n][rows][cols/32]: the bit-plane format of [PW1]          */
+  PW_LAYOUT_TILED_GATE_UP = 1, /* the FFN kernel's layout for a gate_up block               */
+  PW_LAYOUT_TILED_DOWN = 2     /* the FFN kernel's layout for a down block                  */
+};
+
 /* Page states of a Weight Page Table entry [PW1]. */
 enum { PW_PAGE_GPU = 0, PW_PAGE_CPU = 1, PW_PAGE_XFER = 2 };
 
@@ -85,15 +92,25 @@ enum { PW_ACT_HIT = 0, PW_ACT_FETCH = 1, PW_ACT_SUBST = 2 };
  * One Weight Page Table entry: one linear block (layer, expert, module) [PW1].
  *   gate_up: rows = 2I, cols = H (rows 0..I-1 gate, rows I..2I-1 up); down: rows = H, cols = I.
  *   rows % 32 == 0, cols % 128 == 0.
- *   planes: uint32 [parent_bits][rows][cols/32]; plane p holds bit (parent_bits-1-p) of every
- *           parent index (plane 0 = most significant); column 32w+j sits at bit j of word w.
- *           Reading the top q planes gives the q-bit index = top q bits of the parent index.
+ *   Bit-planes: plane p holds bit (parent_bits-1-p) of every parent index (plane 0 = most
+ *   significant), so the top q planes give the q-bit index = top q bits of the parent index.
+ *   In PW_LAYOUT_ROWS a plane is uint32 [rows][cols/32] and column 32w+j sits at bit j of
+ *   word w.  The FFN reads the same words rearranged so that everything one CTA needs for a
+ *   32-row tile and a 1024-column stage is one contiguous run, most significant plane first:
+ *     tile t, row i of the tile:  PW_LAYOUT_TILED_DOWN    -> block row 32t + i;
+ *                                 PW_LAYOUT_TILED_GATE_UP -> gate row 16t + i for i < 16,
+ *                                                            up row I + 16t + (i - 16) otherwise;
+ *     stage s = words 32s .. 32s + ws - 1 of each row, ws = min(32, cols/32 - 32s);
+ *     word w = 32s + 2j + h of plane p, row i of tile t sits at uint32 index
+ *       t * (n * 32 * cols/32) + s * (n * 32 * 32) + p * (32 * ws) + j * 64 + i * 2 + h
+ *     (n = parent_bits).  Reading the top q planes of (t, s) reads the first q * 32 * ws words
+ *     of that run.  `layout` holds PW_LAYOUT_TILED_GATE_UP or PW_LAYOUT_TILED_DOWN; the
+ *     forward checks it against the module.  `planes` is 16-byte aligned.
  *   lut[b]: fp16 [rows][1<<b] for every b in [min_bits, parent_bits] (NULL otherwise);
  *           weight(r, c) at bitwidth q = lut[q][r][top q bits of idx(r, c)].
  *   committed_bits (q_i) is read once per forward call; desired_bits (d_i) is stored for a
  *   planner and ignored by the kernels.
- *   tma_desc: filled by pw_block_prepare() (a TMA tensor-map descriptor over `planes`); the
- *   entry must sit at a 64-byte aligned address on the device.
+ *   The entry must sit at a 64-byte aligned address on the device.
  * sizeof(pw_block) == 256.
  */
 typedef struct pw_block {
@@ -104,11 +121,11 @@ typedef struct pw_block {
   uint8_t desired_bits;
   uint8_t committed_bits;
   uint8_t state;
-  uint8_t reserved0[3];
+  uint8_t layout;
+  uint8_t reserved0[2];
   const uint32_t* planes;
   const uint16_t* lut[9];
-  uint8_t reserved1[32];
-  uint8_t tma_desc[128];
+  uint8_t reserved1[160];
 } pw_block;
 
 /* The Weight Page Table: device-resident; blocks[(layer * num_experts + e) * 2 + module]. */
@@ -128,21 +145,22 @@ typedef struct pw_route_cfg {
 } pw_route_cfg;
 
 /* ---------------------------------------------------------------------------------------
- * pw_block_prepare (host only, no GPU work): validates a host copy of a block entry and
- * encodes its TMA descriptor.  Call after setting rows/cols/parent_bits/min_bits/planes/lut
- * and before copying the entry to the device.  Returns PW_ERR_INVALID_ARG for a bad shape,
- * bitwidth range, missing LUT or misaligned pointer, PW_ERR_CUDA if the driver's
- * tensor-map encoder is unavailable.
+ * pw_block_prepare (host only, no GPU work): validates a host copy of a block entry before
+ * it is copied to the device.  Returns PW_ERR_INVALID_ARG for a bad shape, bitwidth range,
+ * layout, missing LUT or misaligned pointer, PW_ERR_UNSUPPORTED for a block too large for
+ * 32-bit row indexing.
  * ------------------------------------------------------------------------------------- */
 pw_status pw_block_prepare(pw_block* blk_host);
 
 /* ---------------------------------------------------------------------------------------
  * pw_pack_bitplanes [PW1]: uint8 parent indices idx[rows][cols] (values < 2^n) into n
- * bit-planes planes[n][rows][cols/32] in the layout of pw_block.  cols % 32 == 0,
- * 1 <= n <= 8.  Bits of idx above n are ignored.  Offline (untimed) step.
+ * bit-planes in `layout` (PW_LAYOUT_*, defined with pw_block).  cols % 32 == 0 for
+ * PW_LAYOUT_ROWS; rows % 32 == 0 and cols % 128 == 0 for the tiled layouts; 1 <= n <= 8.
+ * Bits of idx above n are ignored.  planes holds n * rows * cols / 32 uint32 words, 16-byte
+ * aligned.  Offline (untimed) step.
  * ------------------------------------------------------------------------------------- */
-pw_status pw_pack_bitplanes(const uint8_t* idx, int rows, int cols, int n, uint32_t* planes,
-                            pw_stream_t stream);
+pw_status pw_pack_bitplanes(const uint8_t* idx, int rows, int cols, int n, int layout,
+                            uint32_t* planes, pw_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------
  * pw_route_topk [LX1]: logits = x W_r^T + bias, then per token the k largest logits in

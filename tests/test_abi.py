@@ -30,15 +30,19 @@ def test_status_strings_and_version(libpw):
 def test_struct_layouts():
     assert ctypes.sizeof(B.pw_block) == 256
     assert B.pw_block.planes.offset == 16 and B.pw_block.lut.offset == 24
-    assert B.pw_block.tma_desc.offset == 128
+    assert B.pw_block.layout.offset == 13 and B.pw_block.reserved1.offset == 96
 
 
 def test_host_argument_checks(libpw):
     cfg = B.pw_route_cfg(k=2, renorm=1, policy=1, threshold=0.15, critical_n=32)
     bad = B.PW_ERR_INVALID_ARG
-    assert B.pw_pack_bitplanes(0, 4, 64, 4, 0) == bad
-    assert B.pw_pack_bitplanes(16, 4, 33, 4, 16) == bad           # ragged columns
-    assert B.pw_pack_bitplanes(16, 4, 64, 9, 16) == bad           # n > 8
+    rows_l, tiled = B.PW_LAYOUT_ROWS, B.PW_LAYOUT_TILED_DOWN
+    assert B.pw_pack_bitplanes(0, 4, 64, 4, rows_l, 0) == bad
+    assert B.pw_pack_bitplanes(16, 4, 33, 4, rows_l, 16) == bad           # ragged columns
+    assert B.pw_pack_bitplanes(16, 4, 64, 9, rows_l, 16) == bad           # n > 8
+    assert B.pw_pack_bitplanes(16, 32, 128, 4, 3, 16) == bad              # unknown layout
+    assert B.pw_pack_bitplanes(16, 48, 128, 4, tiled, 16) == bad          # rows % 32
+    assert B.pw_pack_bitplanes(16, 32, 96, 4, tiled, 16) == bad           # cols % 128
     assert B.pw_route_topk(16, 16, 0, 0, 64, 8, cfg, 16, 16, 16) == bad      # T = 0
     assert B.pw_route_topk(16, 16, 0, 4, 64, 2000, cfg, 16, 16, 16) == bad   # E too large
     cfg.k = 9
@@ -69,3 +73,9 @@ def test_block_prepare_rejects_bad_blocks(libpw):
         blk.lut[b] = 4096 * (b + 1)
     blk.committed_bits = 2
     assert B.pw_block_prepare(blk) == B.PW_ERR_INVALID_ARG                 # q below min_bits
+    blk.committed_bits = 5
+    assert B.pw_block_prepare(blk) == B.PW_ERR_INVALID_ARG                 # rows layout
+    blk.layout = B.PW_LAYOUT_TILED_GATE_UP
+    assert B.pw_block_prepare(blk) == B.PW_OK                              # host-only check
+    blk.planes = 4096 + 8
+    assert B.pw_block_prepare(blk) == B.PW_ERR_INVALID_ARG                 # planes alignment

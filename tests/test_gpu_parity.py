@@ -31,16 +31,43 @@ def _stream(torch):
 
 
 # ------------------------------------------------------------------ K0 pack
+def tiled_reference(planes, layout):
+    """The tiled arrangement of [n][rows][words] bit-planes, built with array reshapes: row
+    tiles of 32 (gate_up: 16 gate rows then the 16 matching up rows), stages of 32 words, and
+    inside a stage [plane][word pair][row][2]."""
+    n, R, W = planes.shape
+    if layout == B.PW_LAYOUT_TILED_GATE_UP:
+        half = R // 2
+        order = np.concatenate([np.r_[16 * t:16 * t + 16, half + 16 * t:half + 16 * t + 16]
+                                for t in range(half // 16)])
+    else:
+        order = np.arange(R)
+    tiles = planes[:, order, :].reshape(n, R // 32, 32, W)
+    out = []
+    for t in range(R // 32):
+        for s0 in range(0, W, 32):
+            blk = tiles[:, t, :, s0:s0 + 32]                      # [n][32][ws]
+            ws = blk.shape[2]
+            out.append(blk.reshape(n, 32, ws // 2, 2).transpose(0, 2, 1, 3).reshape(-1))
+    return np.concatenate(out)
+
+
 @pytest.mark.parametrize("rows,cols,n", [(32, 128, 4), (96, 4096, 8), (64, 1408, 8), (7, 96, 3)])
 def test_pack_bit_exact(torch_dev, rows, cols, n):
     torch, dev = torch_dev
     idx = random_indices(rows, cols, n, seed=rows + cols)
     idx_d = torch.from_numpy(idx).to(dev)
-    planes = torch.full((n, rows, cols // 32), -1, dtype=torch.int32, device=dev)
-    B.check(B.pw_pack_bitplanes(idx_d.data_ptr(), rows, cols, n, planes.data_ptr(),
-                                _stream(torch)))
-    got = planes.cpu().numpy().view(np.uint32)
-    assert np.array_equal(got, obp.pack_bitplanes(idx, n))
+    ref = obp.pack_bitplanes(idx, n)
+    layouts = [B.PW_LAYOUT_ROWS]
+    if rows % 32 == 0 and cols % 128 == 0:
+        layouts += [B.PW_LAYOUT_TILED_GATE_UP, B.PW_LAYOUT_TILED_DOWN]
+    for layout in layouts:
+        planes = torch.full((n * rows * (cols // 32),), -1, dtype=torch.int32, device=dev)
+        B.check(B.pw_pack_bitplanes(idx_d.data_ptr(), rows, cols, n, layout, planes.data_ptr(),
+                                    _stream(torch)))
+        got = planes.cpu().numpy().view(np.uint32)
+        want = ref.reshape(-1) if layout == B.PW_LAYOUT_ROWS else tiled_reference(ref, layout)
+        assert np.array_equal(got, want), f"layout {layout}"
     assert B.pw_get_status(_stream(torch)) == B.PW_OK
 
 
