@@ -237,7 +237,13 @@ pw_status pw_route_topk(const uint16_t* x_bf16, const float* Wr, const float* bi
   }
   if (launch_status() != PW_OK) return PW_ERR_CUDA;
   if (fuse_k) return PW_OK;
-  pw::topk_kernel<<<(T + 7) / 8, 256, 0, st>>>(logits, T, E, cfg->k, cfg->renorm, idx, gate);
+  const int tg = (T + 7) / 8;
+  if (E <= 32) pw::topk_kernel<1><<<tg, 256, 0, st>>>(logits, T, E, cfg->k, cfg->renorm, idx, gate);
+  else if (E <= 64) pw::topk_kernel<2><<<tg, 256, 0, st>>>(logits, T, E, cfg->k, cfg->renorm, idx, gate);
+  else if (E <= 128) pw::topk_kernel<4><<<tg, 256, 0, st>>>(logits, T, E, cfg->k, cfg->renorm, idx, gate);
+  else if (E <= 256) pw::topk_kernel<8><<<tg, 256, 0, st>>>(logits, T, E, cfg->k, cfg->renorm, idx, gate);
+  else if (E <= 512) pw::topk_kernel<16><<<tg, 256, 0, st>>>(logits, T, E, cfg->k, cfg->renorm, idx, gate);
+  else pw::topk_kernel<32><<<tg, 256, 0, st>>>(logits, T, E, cfg->k, cfg->renorm, idx, gate);
   return launch_status();
 }
 
@@ -251,8 +257,18 @@ pw_status pw_substitute(const float* logits, int32_t* idx, const float* gate,
       cfg->policy != PW_POLICY_FIRST_CHOICE)
     return PW_ERR_INVALID_ARG;
   if (cfg->threshold != cfg->threshold) return PW_ERR_INVALID_ARG;  // NaN
-  pw::substitute_kernel<<<(T + 7) / 8, 256, 0, as_cuda(stream)>>>(
-      logits, idx, gate, resident, T, E, cfg->k, cfg->policy, cfg->threshold, action, mass);
+  const dim3 g((T + 7) / 8), b(256);
+  cudaStream_t st = as_cuda(stream);
+#define PW_SUBST(PL)                                                                          \
+  pw::substitute_kernel<PL><<<g, b, 0, st>>>(logits, idx, gate, resident, T, E, cfg->k,      \
+                                             cfg->policy, cfg->threshold, action, mass)
+  if (E <= 32) PW_SUBST(1);
+  else if (E <= 64) PW_SUBST(2);
+  else if (E <= 128) PW_SUBST(4);
+  else if (E <= 256) PW_SUBST(8);
+  else if (E <= 512) PW_SUBST(16);
+  else PW_SUBST(32);
+#undef PW_SUBST
   return launch_status();
 }
 
@@ -262,8 +278,17 @@ pw_status pw_remap(const float* logits, int32_t* idx, const float* gate, int T, 
   if (T < 1 || T > PW_MAX_TOKENS || E < 1 || E > PW_MAX_EXPERTS || !cfg_ok(cfg, E))
     return PW_ERR_INVALID_ARG;
   if (cfg->critical_n < 0 || static_cast<long long>(T) * cfg->k > 8192) return PW_ERR_INVALID_ARG;
-  pw::remap_kernel<<<1, 1024, 0, as_cuda(stream)>>>(logits, idx, gate, T, E, cfg->k,
-                                                    cfg->critical_n, critical);
+  cudaStream_t st = as_cuda(stream);
+#define PW_REMAP(PL)                                                                          \
+  pw::remap_kernel<PL><<<1, 1024, 0, st>>>(logits, idx, gate, T, E, cfg->k, cfg->critical_n, \
+                                           critical)
+  if (E <= 32) PW_REMAP(1);
+  else if (E <= 64) PW_REMAP(2);
+  else if (E <= 128) PW_REMAP(4);
+  else if (E <= 256) PW_REMAP(8);
+  else if (E <= 512) PW_REMAP(16);
+  else PW_REMAP(32);
+#undef PW_REMAP
   return launch_status();
 }
 

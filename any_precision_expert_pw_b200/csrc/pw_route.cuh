@@ -13,7 +13,6 @@ namespace pw {
 
 constexpr int kRouteExpertsPerCta = 8;
 constexpr int kRouteThreads = 256;
-constexpr int kMaxPerLane = PW_MAX_EXPERTS / 32;
 
 __device__ __forceinline__ double bf16lo(uint32_t v) {
   return static_cast<double>(__uint_as_float(v << 16));
@@ -25,25 +24,27 @@ __device__ __forceinline__ double bf16hi(uint32_t v) {
 // One warp, one token: top-k by (logit desc, index asc) over l[0..E), softmax over all E in
 // float64, gates rounded once (renormalised over the k when asked).  Every exp is taken once
 // (float64 exp has a long latency): the selected experts' probabilities are read back from the
-// lane that holds them.
+// lane that holds them.  PL = elements per lane (E <= 32 * PL), so the code is no larger than
+// E needs (a cold kernel fetches every instruction it runs from memory).
+template <int PL>
 __device__ __forceinline__ void topk_warp(const float* l, int E, int k, int renorm,
                                           int32_t* __restrict__ idx_out,
                                           float* __restrict__ gate_out) {
   const int lane = threadIdx.x & 31;
-  float v[kMaxPerLane];
+  float v[PL];
   float mx = -INFINITY;
 #pragma unroll
-  for (int i = 0; i < kMaxPerLane; ++i) {
+  for (int i = 0; i < PL; ++i) {
     const int e = lane + 32 * i;
     v[i] = (e < E) ? l[e] : -INFINITY;
     mx = fmaxf(mx, v[i]);
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-  double ex[kMaxPerLane];
+  double ex[PL];
   double z = 0.0;
 #pragma unroll
-  for (int i = 0; i < kMaxPerLane; ++i) {
+  for (int i = 0; i < PL; ++i) {
     ex[i] = 0.0;
     if (lane + 32 * i < E) {
       ex[i] = exp(static_cast<double>(v[i]) - static_cast<double>(mx));
@@ -59,7 +60,7 @@ __device__ __forceinline__ void topk_warp(const float* l, int E, int k, int reno
     int bi = -1;
     double be = 0.0;
 #pragma unroll
-    for (int i = 0; i < kMaxPerLane; ++i) {
+    for (int i = 0; i < PL; ++i) {
       const int e = lane + 32 * i;
       if (e < E && !((taken >> i) & 1u) && (bi < 0 || v[i] > bv)) {
         bv = v[i];
@@ -188,30 +189,34 @@ __global__ void __launch_bounds__(kRouteThreads) router_logits_kernel(
   if (fuse_k > 0) {
     __syncthreads();
     for (int t = warp; t < nt; t += kRouteThreads / 32)
-      topk_warp(lsm[t], E, fuse_k, renorm, idx + static_cast<size_t>(t0 + t) * fuse_k,
+      topk_warp<1>(lsm[t], E, fuse_k, renorm, idx + static_cast<size_t>(t0 + t) * fuse_k,
                 gate + static_cast<size_t>(t0 + t) * fuse_k);
   }
 }
 
-// One warp per token: top-k of a logits row in global memory.
+// One warp per token: top-k of a logits row in global memory (E <= 32 * PL).
+template <int PL>
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E,
                                                    int k, int renorm, int32_t* __restrict__ idx,
                                                    float* __restrict__ gate) {
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
-  topk_warp(logits + static_cast<size_t>(t) * E, E, k, renorm, idx + static_cast<size_t>(t) * k,
+  topk_warp<PL>(logits + static_cast<size_t>(t) * E, E, k, renorm, idx + static_cast<size_t>(t) * k,
             gate + static_cast<size_t>(t) * k);
 }
 
-// A token's logits row held by one warp: element e = lane + 32 i in v[i] (-inf past E).
+// A token's logits row held by one warp: element e = lane + 32 i in v[i] (-inf past E),
+// E <= 32 * PL.
+template <int PL>
 struct WarpRow {
-  float v[kMaxPerLane];
+  float v[PL];
 };
 
-__device__ __forceinline__ void load_row(const float* __restrict__ l, int E, WarpRow& r) {
+template <int PL>
+__device__ __forceinline__ void load_row(const float* __restrict__ l, int E, WarpRow<PL>& r) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
-  for (int i = 0; i < kMaxPerLane; ++i) {
+  for (int i = 0; i < PL; ++i) {
     const int e = lane + 32 * i;
     r.v[i] = (e < E) ? l[e] : -INFINITY;
   }
@@ -228,13 +233,14 @@ __device__ __forceinline__ uint32_t lane_set(const int* cur, int k) {
 
 // Highest-logit expert e with bit (e >> 5) of this lane's `allowed` set and e not in `chosen`
 // (ties: lower index); -1 if none.
-__device__ __forceinline__ int best_candidate(const WarpRow& r, uint32_t allowed, uint32_t chosen,
-                                              int E) {
+template <int PL>
+__device__ __forceinline__ int best_candidate(const WarpRow<PL>& r, uint32_t allowed,
+                                              uint32_t chosen, int E) {
   const int lane = threadIdx.x & 31;
   float bv = -INFINITY;
   int bi = -1;
 #pragma unroll
-  for (int i = 0; i < kMaxPerLane; ++i) {
+  for (int i = 0; i < PL; ++i) {
     const int e = lane + 32 * i;
     if (e < E && ((allowed >> i) & 1u) && !((chosen >> i) & 1u) && (bi < 0 || r.v[i] > bv)) {
       bv = r.v[i];
@@ -252,6 +258,7 @@ __device__ __forceinline__ void swap_chosen(uint32_t& chosen, int old_e, int new
   if ((new_e & 31) == lane) chosen |= 1u << (new_e >> 5);
 }
 
+template <int PL>
 __global__ void __launch_bounds__(256) substitute_kernel(
     const float* __restrict__ logits, int32_t* __restrict__ idx, const float* __restrict__ gate,
     const uint8_t* __restrict__ resident, int T, int E, int k, int policy, float threshold,
@@ -269,11 +276,11 @@ __global__ void __launch_bounds__(256) substitute_kernel(
     if (lane == 0) set_status(PW_ERR_BAD_EXPERT);
     return;
   }
-  WarpRow row;
+  WarpRow<PL> row;
   load_row(logits + static_cast<size_t>(t) * E, E, row);
   uint32_t res = 0;
 #pragma unroll
-  for (int i = 0; i < kMaxPerLane; ++i) {
+  for (int i = 0; i < PL; ++i) {
     const int e = lane + 32 * i;
     if (e < E && resident[e]) res |= 1u << i;
   }
@@ -311,7 +318,8 @@ __global__ void __launch_bounds__(256) substitute_kernel(
   }
 }
 
-// Single CTA: batch gate sums, critical set, then one warp per token remaps.
+// Single CTA: batch gate sums, critical set, then one warp per token remaps (E <= 32 * PL).
+template <int PL>
 __global__ void __launch_bounds__(1024) remap_kernel(const float* __restrict__ logits,
                                                      int32_t* __restrict__ idx,
                                                      const float* __restrict__ gate, int T, int E,
@@ -369,14 +377,14 @@ __global__ void __launch_bounds__(1024) remap_kernel(const float* __restrict__ l
   const int warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
   uint32_t crit_bits = 0;
 #pragma unroll
-  for (int i = 0; i < kMaxPerLane; ++i) {
+  for (int i = 0; i < PL; ++i) {
     const int e = lane + 32 * i;
     if (e < E && crit[e]) crit_bits |= 1u << i;
   }
   for (int t = warp; t < T; t += nw) {
     int cur[PW_MAX_TOPK];
     for (int j = 0; j < k; ++j) cur[j] = idx[static_cast<size_t>(t) * k + j];
-    WarpRow row;
+    WarpRow<PL> row;
     load_row(logits + static_cast<size_t>(t) * E, E, row);
     uint32_t chosen = lane_set(cur, k);
     for (int s = 1; s < k; ++s) {
