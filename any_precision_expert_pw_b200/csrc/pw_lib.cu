@@ -104,9 +104,6 @@ static __device__ __align__(256) uint8_t g_static_ws[PW_STATIC_WORKSPACE_BYTES];
 void* g_static_ws_addr[kMaxDevices] = {};
 std::mutex g_static_ws_mu;
 
-bool cfg_ok(const pw_route_cfg* cfg, int E) {
-  return cfg && cfg->k >= 1 && cfg->k <= PW_MAX_TOPK && cfg->k <= E;
-}
 
 // k-slices for the down projection: fill the GPU in whole waves of work items, with at least
 // two 1024-column stages per slice.
@@ -210,85 +207,6 @@ pw_status pw_pack_bitplanes(const uint8_t* idx, int rows, int cols, int n, int l
   const int grid = static_cast<int>(blocks < 65535LL * 16 ? blocks : 65535LL * 16);
   pw::pack_bitplanes_kernel<<<grid, 256, 0, as_cuda(stream)>>>(idx, rows, cols, n, layout,
                                                                 planes);
-  return launch_status();
-}
-
-pw_status pw_route_topk(const uint16_t* x_bf16, const float* Wr, const float* bias, int T, int H,
-                        int E, const pw_route_cfg* cfg, float* logits, int32_t* idx, float* gate,
-                        pw_stream_t stream) {
-  if (!x_bf16 || !Wr || !logits || !idx || !gate) return PW_ERR_INVALID_ARG;
-  if (T < 1 || T > PW_MAX_TOKENS || E < 1 || E > PW_MAX_EXPERTS || H < 1 || !cfg_ok(cfg, E))
-    return PW_ERR_INVALID_ARG;
-  DeviceInfo* di = nullptr;
-  if (device_info(&di) != PW_OK) return PW_ERR_CUDA;
-  const int e_tiles = (E + pw::kRouteExpertsPerCta - 1) / pw::kRouteExpertsPerCta;
-  const int t_tiles_target = std::max(1, (2 * di->sms + e_tiles - 1) / e_tiles);
-  int tt = (T + t_tiles_target - 1) / t_tiles_target;
-  tt = tt <= 1 ? 1 : tt <= 2 ? 2 : 4;
-  const int vec = (H % 8 == 0) && (reinterpret_cast<uintptr_t>(x_bf16) % 16 == 0) &&
-                  (reinterpret_cast<uintptr_t>(Wr) % 16 == 0);
-  const dim3 g1(e_tiles, (T + tt - 1) / tt);
-  const int fuse_k = (e_tiles == 1) ? cfg->k : 0;  // the whole E in one CTA: top-k fused
-  cudaStream_t st = as_cuda(stream);
-  switch (tt) {
-    case 1: pw::router_logits_kernel<1><<<g1, pw::kRouteThreads, 0, st>>>(x_bf16, Wr, bias, T, H, E, vec, logits, fuse_k, cfg->renorm, idx, gate); break;
-    case 2: pw::router_logits_kernel<2><<<g1, pw::kRouteThreads, 0, st>>>(x_bf16, Wr, bias, T, H, E, vec, logits, fuse_k, cfg->renorm, idx, gate); break;
-    default: pw::router_logits_kernel<4><<<g1, pw::kRouteThreads, 0, st>>>(x_bf16, Wr, bias, T, H, E, vec, logits, fuse_k, cfg->renorm, idx, gate); break;
-  }
-  if (launch_status() != PW_OK) return PW_ERR_CUDA;
-  if (fuse_k) return PW_OK;
-  const int tg = (T + 7) / 8;
-  if (E <= 32) pw::topk_kernel<1><<<tg, 256, 0, st>>>(logits, T, E, cfg->k, cfg->renorm, idx, gate);
-  else if (E <= 64) pw::topk_kernel<2><<<tg, 256, 0, st>>>(logits, T, E, cfg->k, cfg->renorm, idx, gate);
-  else if (E <= 128) pw::topk_kernel<4><<<tg, 256, 0, st>>>(logits, T, E, cfg->k, cfg->renorm, idx, gate);
-  else if (E <= 256) pw::topk_kernel<8><<<tg, 256, 0, st>>>(logits, T, E, cfg->k, cfg->renorm, idx, gate);
-  else if (E <= 512) pw::topk_kernel<16><<<tg, 256, 0, st>>>(logits, T, E, cfg->k, cfg->renorm, idx, gate);
-  else pw::topk_kernel<32><<<tg, 256, 0, st>>>(logits, T, E, cfg->k, cfg->renorm, idx, gate);
-  return launch_status();
-}
-
-pw_status pw_substitute(const float* logits, int32_t* idx, const float* gate,
-                        const uint8_t* resident, int T, int E, const pw_route_cfg* cfg,
-                        uint8_t* action, float* mass, pw_stream_t stream) {
-  if (!logits || !idx || !gate || !resident) return PW_ERR_INVALID_ARG;
-  if (T < 1 || T > PW_MAX_TOKENS || E < 1 || E > PW_MAX_EXPERTS || !cfg_ok(cfg, E))
-    return PW_ERR_INVALID_ARG;
-  if (cfg->policy != PW_POLICY_FETCH_ALL && cfg->policy != PW_POLICY_THRESHOLD &&
-      cfg->policy != PW_POLICY_FIRST_CHOICE)
-    return PW_ERR_INVALID_ARG;
-  if (cfg->threshold != cfg->threshold) return PW_ERR_INVALID_ARG;  // NaN
-  const dim3 g((T + 7) / 8), b(256);
-  cudaStream_t st = as_cuda(stream);
-#define PW_SUBST(PL)                                                                          \
-  pw::substitute_kernel<PL><<<g, b, 0, st>>>(logits, idx, gate, resident, T, E, cfg->k,      \
-                                             cfg->policy, cfg->threshold, action, mass)
-  if (E <= 32) PW_SUBST(1);
-  else if (E <= 64) PW_SUBST(2);
-  else if (E <= 128) PW_SUBST(4);
-  else if (E <= 256) PW_SUBST(8);
-  else if (E <= 512) PW_SUBST(16);
-  else PW_SUBST(32);
-#undef PW_SUBST
-  return launch_status();
-}
-
-pw_status pw_remap(const float* logits, int32_t* idx, const float* gate, int T, int E,
-                   const pw_route_cfg* cfg, uint8_t* critical, pw_stream_t stream) {
-  if (!logits || !idx || !gate) return PW_ERR_INVALID_ARG;
-  if (T < 1 || T > PW_MAX_TOKENS || E < 1 || E > PW_MAX_EXPERTS || !cfg_ok(cfg, E))
-    return PW_ERR_INVALID_ARG;
-  if (cfg->critical_n < 0 || static_cast<long long>(T) * cfg->k > 8192) return PW_ERR_INVALID_ARG;
-  cudaStream_t st = as_cuda(stream);
-#define PW_REMAP(PL)                                                                          \
-  pw::remap_kernel<PL><<<1, 1024, 0, st>>>(logits, idx, gate, T, E, cfg->k, cfg->critical_n, \
-                                           critical)
-  if (E <= 32) PW_REMAP(1);
-  else if (E <= 64) PW_REMAP(2);
-  else if (E <= 128) PW_REMAP(4);
-  else if (E <= 256) PW_REMAP(8);
-  else if (E <= 512) PW_REMAP(16);
-  else PW_REMAP(32);
-#undef PW_REMAP
   return launch_status();
 }
 
@@ -428,3 +346,6 @@ pw_status pw_get_status(pw_stream_t stream) {
 }
 
 }  // extern "C"
+
+// Routing-side entry points (pw_route_topk, pw_substitute, pw_remap): same translation unit.
+#include "pw_route_api.cuh"
