@@ -146,17 +146,51 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sms)}
 
 
-def dist_init(n_gpus):
-    import torch
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
+class Replicas:
+    """N independent replicas of the layer, one process per GPU (torchrun's RANK / WORLD_SIZE /
+    LOCAL_RANK / MASTER_* environment).  The process group carries no layer data: only the
+    barriers around the timed region and the max over ranks of the measured times.  backend
+    "nccl" on GPUs; "gloo" runs the same bookkeeping on CPU processes."""
+
+    def __init__(self, backend="nccl", timeout_s=120):
+        import torch
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.backend = backend
+        self.device = torch.device(f"cuda:{self.local}") if backend == "nccl" else torch.device("cpu")
+        if self.world > 1:
+            import torch.distributed as dist
+            kw = {"timeout": datetime.timedelta(seconds=timeout_s)}
+            if backend == "nccl":
+                torch.cuda.set_device(self.local)
+                kw["device_id"] = self.device
+            dist.init_process_group(backend, **kw)
+
+    def barrier(self):
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max_over_ranks(self, v):
+        if self.world == 1:
+            return v
+        import torch
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device(f"cuda:{local}"))
-    return world, rank, local
+        t = torch.tensor([v], dtype=torch.float64, device=self.device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+def replica_value(world, tokens_per_replica, step_ms):
+    """Whole-job tokens/s: every replica processes its own batch in the (max) step time."""
+    return world * tokens_per_replica / (step_ms * 1e-3)
 
 
 def oracle_step(L, frac):
@@ -251,7 +285,8 @@ def run_pw(args):
     from any_precision_expert_pw_b200.device_layer import DeviceLayer
     from any_precision_expert_pw_b200.inputs import POLICY_NONE, make_layer
 
-    world, rank, local = dist_init(args.gpus)
+    rep = Replicas("nccl")
+    world, rank, local = rep.world, rep.rank, rep.local
     dev = torch.device(f"cuda:{local}")
     torch.cuda.set_device(dev)
     cfg, T = workload(args)
@@ -302,16 +337,8 @@ def run_pw(args):
     def mean_ms(evs):
         return sum(a.elapsed_time(b) for a, b in evs) / len(evs)
 
-    def barrier():
-        if world > 1:
-            torch.distributed.barrier()
-
-    def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        return float(t.item())
+    barrier = rep.barrier
+    max_over_ranks = rep.max_over_ranks
 
     timed(g_step, args.warmup)
     torch.cuda.synchronize(dev)
@@ -364,7 +391,7 @@ def run_pw(args):
     peak, peak_kind = read_peaks()
     achieved = b_ffn / (ffn_ms * 1e-3) / 1e9
     traffic = recorded_traffic()
-    value = world * T / (step_ms * 1e-3)
+    value = replica_value(world, T, step_ms)
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
@@ -384,7 +411,7 @@ def run_pw(args):
                      "frac": achieved / peak, "traffic": traffic,
                      "kernel": "pw_moe_anyprec_forward (grouping + gate_up + down + combine)",
                      "peak_kind": f"{peak_kind} copy bandwidth (burst)"},
-        "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": replica_value(world, T, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(T * cfg.H * 2), "d2h_bytes_per_step": int(T * cfg.H * 4),
                 "ms_per_step": e2e_ms, "path": "pinned x -> pw_route_topk -> "
                 "pw_moe_anyprec_forward -> pinned y, direct calls (no graph)"},
@@ -398,9 +425,7 @@ def run_pw(args):
     if rank == 0:
         print(json.dumps(out), flush=True)
     del g_step, g_ffn
-    if world > 1:
-        torch.distributed.barrier()
-        torch.distributed.destroy_process_group()
+    rep.close()
 
 
 def main():
