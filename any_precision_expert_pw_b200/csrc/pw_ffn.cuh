@@ -54,8 +54,8 @@ constexpr int kPlaneBytes = kRows * kStageWords * 4;     // one plane of a full 
 constexpr int kStagePlaneBytes = PW_MAX_BITS * kPlaneBytes;
 constexpr int kLutBytes = 256 * 256;                     // 2^8 entries x 256-byte stride
 constexpr int kMaxKSlices = 8;
-constexpr int kDescRing = 4;
-constexpr int kPrefetchItems = 2;  // down: items per CTA prefetched into L2 before h is ready
+constexpr int kDescRing = 8;    // item descriptors in flight (LUT warps -> every other role)
+constexpr int kLutBarrier = 1;  // named barrier of the four LUT warps
 
 // The kernel's dynamic shared memory, named directly (not through a pointer) wherever the
 // decode loop indexes it, so every table gather is one load with a constant base folded in.
@@ -78,9 +78,9 @@ struct Layout {
   static constexpr int kOffRed = kOffStages + kStages * kStageBytes;
   static constexpr int kRedBytes = 2 * kDecodeWarps * NTP * 32 * 4;
   static constexpr int kOffDesc = kOffRed + kRedBytes;
-  static constexpr int kDescBytes = kDescRing * 48;
+  static constexpr int kDescBytes = kDescRing * 80;
   static constexpr int kOffBar = kOffDesc + kDescBytes;
-  static constexpr int kBarBytes = (2 * kStages + 8) * 8 + 32;
+  static constexpr int kBarBytes = (2 * kStages + 8 + 2 * kDescRing) * 8 + 32;
   static constexpr int kSmem = kOffBar + kBarBytes;
   static_assert(kStageBytes % 128 == 0 && kOffStages % 128 == 0, "stage alignment");
   static_assert(kSmem <= 227 * 1024, "shared memory budget");
@@ -109,13 +109,17 @@ struct Params {
   float* out;        // gate_up: h [pos][ld_out] (xslot order); down: [kslice][pos][ld_out]
   int ld_out;
   long long out_slice;  // elements between k-slices of `out`
+  int* sched;           // work counter (zero at launch): items after each CTA's first one
 };
 
-// What the producer tells the LUT and decode warps about an item (shared-memory rings).
+// One work item as every warp role sees it: written once by LUT warp 0 into a shared-memory
+// ring; item < 0 marks the end of this CTA's work.
 struct Desc {
-  int valid, status, q, te, pos0, tile, ks, s0, s1, pad0, pad1, pad2;
+  const uint32_t* planes;  // the tile's run of stages (tiled layout)
+  const uint16_t* lut;     // the block's q-bit LUT
+  int item, valid, status, q, n, te, pos0, tile, ks, s0, s1, segA, segB, pad0, pad1, pad2;
 };
-static_assert(sizeof(Desc) == 48, "descriptor size");
+static_assert(sizeof(Desc) == 80, "descriptor size");
 
 struct Item {
   const pw_block* blk;
@@ -425,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
   uint64_t* lut_free = lut_ready + 2;         // [2] table released (decode -> LUT warps)
   uint64_t* red_full = lut_free + 2;          // [2] partial sums written (decode -> reducer)
   uint64_t* red_free = red_full + 2;          // [2] partial sums consumed (reducer -> decode)
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(red_free + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(red_free + 2 + 2 * kDescRing);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (smem_u32(smem) & 127) {  // stage buffers and tables assume 128-byte alignment
@@ -443,6 +447,10 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
       mbar_init(&red_full[b], kDecodeWarps);
       mbar_init(&red_free[b], 1);
     }
+    for (int r = 0; r < kDescRing; ++r) {
+      mbar_init(&red_free[2 + r], 1);              // desc_full: written by LUT warp 0
+      mbar_init(&red_free[2 + kDescRing + r], 2);  // desc_free: read by producer and reducer
+    }
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -455,26 +463,31 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
   const int n_items = p.meta[0] * p.tiles * p.kslices;
   const int words_total = p.cols / 32;
 
+  uint64_t* const desc_full = red_free + 2;  // [kDescRing] descriptor written (LUT warp 0)
+  uint64_t* const desc_free = desc_full + kDescRing;  // [kDescRing] read by producer + reducer
+
   if (warp == kProducerWarp) {
     // ---------------- producer: one thread streams every stage ----------------
     if (lane != 0) return;
     if (p.mode == MODE_DOWN) {
-      // while the gate_up grid finishes: this CTA's first items' planes into L2, then wait for h
-      for (int item = blockIdx.x, n = 0; item < n_items && n < kPrefetchItems;
-           item += gridDim.x, ++n) {
-        const Item cur = resolve(p, item);
-        if (!cur.valid) continue;
-        for (int s = cur.s0; s < cur.s1; ++s) {
-          const int ws = min(kStageWords, words_total - s * kStageWords);
-          prefetch_l2(cur.planes + static_cast<size_t>(s) * cur.n * kRows * kStageWords,
-                      cur.q * ws * kRows * 4);
-        }
+      // while the gate_up grid finishes: this CTA's first item's planes into L2, then wait for h
+      if (static_cast<int>(blockIdx.x) < n_items) {
+        const Item cur = resolve(p, blockIdx.x);
+        if (cur.valid)
+          for (int s = cur.s0; s < cur.s1; ++s) {
+            const int ws = min(kStageWords, words_total - s * kStageWords);
+            prefetch_l2(cur.planes + static_cast<size_t>(s) * cur.n * kRows * kStageWords,
+                        cur.q * ws * kRows * 4);
+          }
       }
       griddep_wait();
     }
     uint32_t g = 0;
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-      const Item cur = resolve(p, item);
+    for (uint32_t j = 0;; ++j) {
+      wait_bar(&desc_full[j % kDescRing], (j / kDescRing) & 1, abort_flag);
+      const Desc cur = cdesc[j % kDescRing];
+      mbar_arrive(&desc_free[j % kDescRing]);
+      if (cur.item < 0 || *abort_flag) break;
       if (!cur.valid) continue;
       for (int ch = 0; ch < cur.te; ch += NTP) {
         const int ntok = min(NTP, cur.te - ch);
@@ -508,8 +521,12 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
   if (warp == kReducerWarp) {
     // ---------------- reducer: sixteen partial sums per row, in warp order ----------------
     uint32_t rc = 0;
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-      const Item it = resolve(p, item);
+    for (uint32_t j = 0;; ++j) {
+      wait_bar(&desc_full[j % kDescRing], (j / kDescRing) & 1, abort_flag);
+      const Desc it = cdesc[j % kDescRing];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&desc_free[j % kDescRing]);
+      if (it.item < 0 || *abort_flag) break;
       if (!it.valid) continue;
       for (int ch = 0; ch < it.te; ch += NTP, ++rc) {
         const int ntok = min(NTP, it.te - ch);
@@ -539,12 +556,55 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
   }
 
   if (warp >= kLutWarp0) {
-    // ---------------- LUT warps: item descriptors and decode tables ----------------
+    // ---------------- LUT warps: the item schedule and the decode tables ----------------
+    // Item 0 of each CTA is blockIdx.x; every later one is taken from the launch's work counter
+    // (gridDim.x + its old value), so CTAs that finish early take more items.  LUT warp 0
+    // resolves each item and publishes its descriptor; all four warps then build its table.
     const int lw = warp - kLutWarp0;
-    uint32_t j = 0;
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++j) {
+    int item = blockIdx.x;
+    for (uint32_t j = 0;; ++j) {
       const uint32_t u = j & 1;
-      const Item it = resolve(p, item);
+      Desc& d = cdesc[j % kDescRing];
+      if (lw == 0) {
+        int next = 0;
+        if (lane == 0 && item < n_items) next = gridDim.x + atomicAdd(p.sched, 1);
+        if (lane == 0) {
+          // the producer and the reducer have read descriptor j - kDescRing from this slot
+          wait_bar(&desc_free[j % kDescRing], ((j / kDescRing) & 1) ^ 1, abort_flag);
+          if (item < n_items) {
+            const Item it = resolve(p, item);
+            d.planes = it.planes;
+            d.lut = it.lut;
+            d.item = item;
+            d.valid = it.valid;
+            d.status = it.status;
+            d.q = it.q;
+            d.n = it.n;
+            d.te = it.te;
+            d.pos0 = it.pos0;
+            d.tile = it.tile;
+            d.ks = it.ks;
+            d.s0 = it.s0;
+            d.s1 = it.s1;
+            d.segA = it.segA;
+            d.segB = it.segB;
+          } else {
+            d.item = -1;
+          }
+          mbar_arrive(&desc_full[j % kDescRing]);
+        }
+        item = __shfl_sync(0xffffffffu, next, 0);
+      }
+      named_sync(kLutBarrier, kLutWarps * 32);  // descriptor j visible to the four LUT warps
+      const Desc it = d;
+      if (it.item < 0 || *abort_flag) {
+        // the decode warps read the end marker; like any item it follows their release of
+        // buffer u (item j - 2), so no barrier phase runs ahead of a waiter
+        wait_bar(&lut_free[u], ((j >> 1) & 1) ^ 1, abort_flag);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&lut_ready[u]);
+        break;
+      }
       LutRegs lr;
       if (it.valid) {
         const int r = lane < kSegRows ? it.segA + lane : it.segB + (lane - kSegRows);
@@ -552,18 +612,6 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
       }
       wait_bar(&lut_free[u], ((j >> 1) & 1) ^ 1, abort_flag);  // decode warps left item j-2
       if (it.valid) store_table(lr, it.q, u, lw, lane);
-      if (lw == 0 && lane == 0) {
-        Desc& d = cdesc[j % kDescRing];
-        d.valid = it.valid;
-        d.status = it.status;
-        d.q = it.q;
-        d.te = it.te;
-        d.pos0 = it.pos0;
-        d.tile = it.tile;
-        d.ks = it.ks;
-        d.s0 = it.s0;
-        d.s1 = it.s1;
-      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&lut_ready[u]);
     }
@@ -573,11 +621,12 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
   // ---------------- decode warps ----------------
   const int tid = threadIdx.x;
   const int ndec = kDecodeWarps * 32;
-  uint32_t g = 0, j = 0, rc = 0;
-  for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++j) {
+  uint32_t g = 0, rc = 0;
+  for (uint32_t j = 0;; ++j) {
     const uint32_t u = j & 1;
     wait_bar(&lut_ready[u], (j >> 1) & 1, abort_flag);
     const Desc d = cdesc[j % kDescRing];
+    if (d.item < 0 || *abort_flag) break;
     if (!d.valid) {
       if (tid == 0) set_status(d.status);
       for (int i = tid; i < d.te * kRows; i += ndec) {

@@ -15,7 +15,7 @@ constexpr int kMaxAssign = 8192;  // T * k handled by the single-CTA grouping st
 // assignment), inv[T*k] (assignment -> grouped position, -1 for an invalid expert id),
 // active[E] (experts with work, ascending), meta[0] = number of active experts (0 when the page
 // table does not match (layer, E)), meta[1] = number of valid assignments, meta[2] = 1 for a
-// mismatched table.
+// mismatched table, meta[4] / meta[5] = 0 (the FFN launches' work counters).
 __device__ __forceinline__ void group_block(const pw_page_table* __restrict__ pt, int layer,
                                             const int32_t* __restrict__ idx, int TK, int E,
                                             int32_t* __restrict__ counts,
@@ -58,6 +58,8 @@ __device__ __forceinline__ void group_block(const pw_page_table* __restrict__ pt
     meta[0] = bad ? 0 : na;
     meta[1] = o;
     meta[2] = bad ? 1 : 0;
+    meta[4] = 0;  // work counters of the gate_up and down launches
+    meta[5] = 0;
   }
   __syncthreads();
   for (int e = tid; e < E; e += blockDim.x) {

@@ -89,7 +89,7 @@ Workspace ws_layout(int T, int k, int E, int H, int I) {
   w.perm = take(4 * TK);
   w.inv = take(4 * TK);
   w.active = take(4 * static_cast<size_t>(E));
-  w.meta = take(16);
+  w.meta = take(32);  // [0] active experts, [1] valid assignments, [2] bad table, [4..5] work counters
   w.X = take(4 * static_cast<size_t>(T) * w.ldx);
   w.Hbuf = take(4 * TK * w.ldh);
   w.O = take(4 * TK * H * static_cast<size_t>(pw::k4::kMaxKSlices));
@@ -270,6 +270,7 @@ pw_status pw_moe_anyprec_forward(const pw_page_table* pt_dev, int layer, int E,
   p.half = I;
   p.tiles = I / pw::k4::kSegRows;
   p.kslices = 1;
+  p.sched = meta + 4;
   p.act = X;
   p.ld_act = w.ldx;
   p.act_map = perm;  // grouped position -> assignment t*k+slot -> token row of X
@@ -287,6 +288,7 @@ pw_status pw_moe_anyprec_forward(const pw_page_table* pt_dev, int layer, int E,
   p.tiles = H / pw::k4::kRows;
   p.kslices = choose_kslices(max_active * p.tiles, (I + pw::k4::kStageCols - 1) / pw::k4::kStageCols,
                              di->sms);
+  p.sched = meta + 5;
   p.act = Hb;
   p.ld_act = w.ldh;
   p.act_map = nullptr;

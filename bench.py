@@ -32,6 +32,7 @@ if ROOT not in sys.path:
 
 METRIC = "MoE decode layer tokens/s and effective weight HBM GB/s (fraction of peak)"
 FALLBACK_HBM_GBS = 6650.0
+SPEC_HBM_GBS = 8000.0          # B200 HBM3e data-sheet figure, for the spec fraction
 WORKLOAD = ("mixtral_8x7b", 1)
 
 
@@ -281,7 +282,7 @@ def run_pw(args):
     import torch
 
     from any_precision_expert_pw_b200 import binding as B
-    from any_precision_expert_pw_b200.accounting import ffn_bytes, layer_bytes
+    from any_precision_expert_pw_b200.accounting import ffn_bytes, layer_bytes, plane_bytes
     from any_precision_expert_pw_b200.device_layer import DeviceLayer
     from any_precision_expert_pw_b200.inputs import POLICY_NONE, make_layer
 
@@ -337,6 +338,9 @@ def run_pw(args):
     def mean_ms(evs):
         return sum(a.elapsed_time(b) for a, b in evs) / len(evs)
 
+    def median_ms(evs):
+        return statistics.median(a.elapsed_time(b) for a, b in evs)
+
     barrier = rep.barrier
     max_over_ranks = rep.max_over_ranks
 
@@ -355,6 +359,7 @@ def run_pw(args):
     t_wall1 = time.perf_counter()
     clk = clocks.stop()
     step_ms = max_over_ranks(mean_ms(evs))
+    step_med_ms = max_over_ranks(median_ms(evs))
 
     # FFN call alone (the dominant kernels): roofline numerator
     timed(g_ffn, args.warmup)
@@ -388,6 +393,7 @@ def run_pw(args):
     used = np.unique(D.idx.cpu().numpy())
     b_layer = layer_bytes(cfg.H, cfg.I, cfg.E, L.q, used, T, bool(np.any(L.bias != 0)))
     b_ffn = ffn_bytes(cfg.H, cfg.I, L.q, used, T)
+    b_planes = plane_bytes(cfg.H, cfg.I, L.q, used)
     peak, peak_kind = read_peaks()
     achieved = b_ffn / (ffn_ms * 1e-3) / 1e9
     traffic = recorded_traffic()
@@ -403,8 +409,11 @@ def run_pw(args):
                    "parallelism": f"replicas{world}" if world > 1 else "single",
                    "l2": "flushed before every step (memset of 2.5x L2, outside the step events)",
                    "timing": "CUDA-graph replay per step, CUDA events on the launching stream"},
+        "ms_per_step_median": step_med_ms,
         "effective_gbs": b_layer / (step_ms * 1e-3) / 1e9,
         "hbm_frac": b_layer / (step_ms * 1e-3) / 1e9 / peak,
+        "hbm_frac_of_spec": b_layer / (step_ms * 1e-3) / 1e9 / SPEC_HBM_GBS,
+        "plane_gbs": b_planes / (step_ms * 1e-3) / 1e9,
         "bytes_per_step": b_layer,
         "ffn_ms": ffn_ms,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
