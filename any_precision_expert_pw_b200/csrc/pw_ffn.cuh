@@ -566,8 +566,6 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
       const uint32_t u = j & 1;
       Desc& d = cdesc[j % kDescRing];
       if (lw == 0) {
-        int next = 0;
-        if (lane == 0 && item < n_items) next = gridDim.x + atomicAdd(p.sched, 1);
         if (lane == 0) {
           // the producer and the reducer have read descriptor j - kDescRing from this slot
           wait_bar(&desc_free[j % kDescRing], ((j / kDescRing) & 1) ^ 1, abort_flag);
@@ -593,7 +591,6 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
           }
           mbar_arrive(&desc_full[j % kDescRing]);
         }
-        item = __shfl_sync(0xffffffffu, next, 0);
       }
       named_sync(kLutBarrier, kLutWarps * 32);  // descriptor j visible to the four LUT warps
       const Desc it = d;
@@ -611,7 +608,12 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
         fetch_table(it.lut + (static_cast<size_t>(r) << it.q), it.q, lw, lr);
       }
       wait_bar(&lut_free[u], ((j >> 1) & 1) ^ 1, abort_flag);  // decode warps left item j-2
+      // claim item j + 1 only now, two items ahead of the decode warps: an item claimed earlier
+      // would sit in this CTA's queue while other CTAs run dry at the end of the launch
+      int next = 0;
+      if (lw == 0 && lane == 0) next = gridDim.x + atomicAdd(p.sched, 1);
       if (it.valid) store_table(lr, it.q, u, lw, lane);
+      if (lw == 0) item = __shfl_sync(0xffffffffu, next, 0);
       __syncwarp();
       if (lane == 0) mbar_arrive(&lut_ready[u]);
     }

@@ -95,6 +95,7 @@ __global__ void __launch_bounds__(kGroupThreads) setup_kernel(
     int I, int ldh, float* __restrict__ Hbuf, int32_t* __restrict__ counts,
     int32_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ inv,
     int32_t* __restrict__ active, int32_t* __restrict__ meta) {
+  griddep_wait();  // launched as a dependent of whatever precedes it in the stream
   griddep_launch();
   if (blockIdx.x == 0) {
     group_block(pt, layer, idx, T * k, E, counts, offsets, perm, inv, active, meta);

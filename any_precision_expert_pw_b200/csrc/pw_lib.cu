@@ -249,10 +249,10 @@ pw_status pw_moe_anyprec_forward(const pw_page_table* pt_dev, int layer, int E,
     const long long conv = (groups + pw::kGroupThreads - 1) / pw::kGroupThreads;
     const int grid = 1 + static_cast<int>(std::min<long long>(std::max(conv, 1LL), 2LL * di->sms));
     const int vec = (reinterpret_cast<uintptr_t>(x_bf16) % 16) == 0;
-    pw::setup_kernel<<<grid, pw::kGroupThreads, 0, st>>>(pt_dev, layer, idx, T, k, E, x_bf16, H,
-                                                          w.ldx, vec, X, I, w.ldh, Hb, counts,
-                                                          offsets, perm, inv, active, meta);
-    if (launch_status() != PW_OK) return PW_ERR_CUDA;
+    if (launch_dependent(pw::setup_kernel, dim3(grid), dim3(pw::kGroupThreads), 0, st, pt_dev,
+                         layer, idx, T, k, E, x_bf16, H, w.ldx, vec, X, I, w.ldh, Hb, counts,
+                         offsets, perm, inv, active, meta) != PW_OK)
+      return PW_ERR_CUDA;
   }
   const int max_active = E < TK ? E : TK;
   pw::k4::Params p;

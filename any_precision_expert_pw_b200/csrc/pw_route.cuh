@@ -89,6 +89,7 @@ __global__ void __launch_bounds__(kRouteThreads) router_logits_kernel(
     const uint16_t* __restrict__ x, const float* __restrict__ Wr, const float* __restrict__ bias,
     int T, int H, int E, int vec, float* __restrict__ logits, int fuse_k, int renorm,
     int32_t* __restrict__ idx, float* __restrict__ gate) {
+  griddep_launch();  // the next kernel (a rewrite or the forward's setup) may be scheduled now
   __shared__ double part[kRouteThreads / 32][kRouteExpertsPerCta][TT];
   __shared__ float lsm[TT][kRouteExpertsPerCta];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
