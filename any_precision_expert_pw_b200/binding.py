@@ -36,7 +36,8 @@ PW_MAX_TOKENS = 4096
 
 # every symbol include/pw.h declares
 EXPORTS = ("pw_block_prepare", "pw_pack_bitplanes", "pw_route_topk", "pw_substitute",
-           "pw_remap", "pw_moe_workspace_bytes", "pw_moe_anyprec_forward",
+           "pw_remap", "pw_affinity_default", "pw_affinity_remap", "pw_moe_workspace_bytes",
+           "pw_moe_anyprec_forward",
            "pw_moe_anyprec_forward_static", "pw_commit_bits", "pw_get_status",
            "pw_status_string", "pw_version")
 PW_STATIC_WORKSPACE_BYTES = 16 << 20
@@ -68,6 +69,12 @@ class pw_route_cfg(ctypes.Structure):
                 ("threshold", ctypes.c_float), ("critical_n", ctypes.c_int32)]
 
 
+class pw_affinity_cfg(ctypes.Structure):
+    _fields_ = [("num_bins", ctypes.c_int32), ("low_bins", ctypes.c_int32),
+                ("bin_width", ctypes.c_double)]
+
+
+assert ctypes.sizeof(pw_affinity_cfg) == 16
 assert ctypes.sizeof(pw_block) == 256 and pw_block.layout.offset == 13
 assert ctypes.sizeof(pw_page_table) == 16 and ctypes.sizeof(pw_route_cfg) == 20
 
@@ -88,6 +95,9 @@ def lib() -> ctypes.CDLL:
         L.pw_route_topk.argtypes = [P, P, P, I, I, I, ctypes.POINTER(pw_route_cfg), P, P, P, S]
         L.pw_substitute.argtypes = [P, P, P, P, I, I, ctypes.POINTER(pw_route_cfg), P, P, S]
         L.pw_remap.argtypes = [P, P, P, I, I, ctypes.POINTER(pw_route_cfg), P, S]
+        L.pw_affinity_default.argtypes = [I, I, ctypes.POINTER(pw_affinity_cfg)]
+        L.pw_affinity_remap.argtypes = [P, P, P, I, I, ctypes.POINTER(pw_route_cfg),
+                                        ctypes.POINTER(pw_affinity_cfg), P, P, S]
         L.pw_moe_workspace_bytes.argtypes = [I, I, I, I, I]
         L.pw_moe_workspace_bytes.restype = Z
         L.pw_moe_anyprec_forward.argtypes = [P, I, I, P, I, I, I, I, P, P, P, P, Z, S]
@@ -147,6 +157,15 @@ def pw_substitute(logits, idx, gate, resident, T, E, cfg, action, mass, stream=0
 
 def pw_remap(logits, idx, gate, T, E, cfg, critical, stream=0) -> int:
     return lib().pw_remap(logits, idx, gate, T, E, _cfg(cfg), critical, stream)
+
+
+def pw_affinity_default(E, k, out) -> int:
+    return lib().pw_affinity_default(E, k, _cfg(out))
+
+
+def pw_affinity_remap(logits, idx, gate, T, E, cfg, acfg, critical, bins, stream=0) -> int:
+    return lib().pw_affinity_remap(logits, idx, gate, T, E, _cfg(cfg), _cfg(acfg), critical,
+                                   bins, stream)
 
 
 def pw_moe_workspace_bytes(T, k, E, H, I) -> int:

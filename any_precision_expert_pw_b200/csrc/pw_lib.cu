@@ -23,6 +23,7 @@ static_assert(offsetof(pw_block, lut) == 24, "pw_block layout");
 static_assert(offsetof(pw_block, layout) == 13, "pw_block layout");
 static_assert(sizeof(pw_page_table) == 16, "pw_page_table layout");
 static_assert(sizeof(pw_route_cfg) == 20, "pw_route_cfg layout");
+static_assert(sizeof(pw_affinity_cfg) == 16, "pw_affinity_cfg layout");
 
 namespace {
 

@@ -319,6 +319,8 @@ __global__ void __launch_bounds__(256) substitute_kernel(
   }
 }
 
+constexpr int kRemapMaxAssign = 8192;  // T * k of the single-CTA batch rewrites
+
 // Single CTA: batch gate sums, critical set, then one warp per token remaps (E <= 32 * PL).
 template <int PL>
 __global__ void __launch_bounds__(1024) remap_kernel(const float* __restrict__ logits,
@@ -329,6 +331,7 @@ __global__ void __launch_bounds__(1024) remap_kernel(const float* __restrict__ l
   __shared__ double S[PW_MAX_EXPERTS];
   __shared__ uint8_t r0[PW_MAX_EXPERTS];
   __shared__ uint8_t crit[PW_MAX_EXPERTS];
+  __shared__ int16_t idx_s[kRemapMaxAssign];  // the assignments, scanned once per expert
   __shared__ int n_r0;
   __shared__ int bad;
   const int tid = threadIdx.x;
@@ -342,18 +345,19 @@ __global__ void __launch_bounds__(1024) remap_kernel(const float* __restrict__ l
   for (int a = tid; a < TK; a += blockDim.x) {
     const int e = idx[a];
     if (e < 0 || e >= E) atomicExch(&bad, 1);
+    idx_s[a] = static_cast<int16_t>(e);
   }
   __syncthreads();
   if (bad) {
     if (tid == 0) set_status(PW_ERR_BAD_EXPERT);
     return;
   }
-  for (int t = tid; t < T; t += blockDim.x) r0[idx[static_cast<size_t>(t) * k]] = 1;
+  for (int t = tid; t < T; t += blockDim.x) r0[idx_s[t * k]] = 1;
   // S_e: float64, ascending (token, slot) order -- one thread per expert scans the batch.
   for (int e = tid; e < E; e += blockDim.x) {
     double s = 0.0;
     for (int a = 0; a < TK; ++a)
-      if (idx[a] == e) s += static_cast<double>(gate[a]);
+      if (idx_s[a] == e) s += static_cast<double>(gate[a]);
     S[e] = s;
   }
   __syncthreads();
@@ -383,6 +387,136 @@ __global__ void __launch_bounds__(1024) remap_kernel(const float* __restrict__ l
     if (e < E && crit[e]) crit_bits |= 1u << i;
   }
   for (int t = warp; t < T; t += nw) {
+    int cur[PW_MAX_TOPK];
+    for (int j = 0; j < k; ++j) cur[j] = idx[static_cast<size_t>(t) * k + j];
+    WarpRow<PL> row;
+    load_row(logits + static_cast<size_t>(t) * E, E, row);
+    uint32_t chosen = lane_set(cur, k);
+    for (int s = 1; s < k; ++s) {
+      if (crit[cur[s]]) continue;
+      const int c = best_candidate(row, crit_bits, chosen, E);
+      if (c >= 0) {
+        swap_chosen(chosen, cur[s], c);
+        cur[s] = c;
+      }
+    }
+    __syncwarp();
+    if (lane == 0)
+      for (int s = 1; s < k; ++s) idx[static_cast<size_t>(t) * k + s] = cur[s];
+  }
+}
+
+// LYNX AffinityBinning (2.1, 2.2): per-token confidence bins from the top-2 logit gap, batch
+// expert scores S_e = sum of 2^bin * gate (float64, ascending (token, slot) order), the critical
+// set from those scores, then the remap of low-affinity tokens (bin < low) as in remap_kernel.
+// One CTA; bins[T] (int32) may be null.
+template <int PL>
+__global__ void __launch_bounds__(1024) affinity_remap_kernel(
+    const float* __restrict__ logits, int32_t* __restrict__ idx, const float* __restrict__ gate,
+    int T, int E, int k, int critical_n, int B, double w, int low,
+    uint8_t* __restrict__ critical, int32_t* __restrict__ bins_out) {
+  __shared__ double S[PW_MAX_EXPERTS];
+  __shared__ uint8_t r0[PW_MAX_EXPERTS];
+  __shared__ uint8_t crit[PW_MAX_EXPERTS];
+  __shared__ uint8_t bin_s[PW_MAX_TOKENS];
+  __shared__ int16_t idx_s[kRemapMaxAssign];
+  __shared__ int n_r0;
+  __shared__ int bad;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
+  const int TK = T * k;
+  if (tid == 0) {
+    n_r0 = 0;
+    bad = 0;
+  }
+  for (int e = tid; e < E; e += blockDim.x) r0[e] = 0;
+  __syncthreads();
+  for (int a = tid; a < TK; a += blockDim.x) {
+    const int e = idx[a];
+    if (e < 0 || e >= E) atomicExch(&bad, 1);
+    idx_s[a] = static_cast<int16_t>(e);
+  }
+  __syncthreads();
+  if (bad) {
+    if (tid == 0) set_status(PW_ERR_BAD_EXPERT);
+    return;
+  }
+  // confidence bins: warp per token, gap between the two largest logits (fp32)
+  for (int t = warp; t < T; t += nw) {
+    WarpRow<PL> row;
+    load_row(logits + static_cast<size_t>(t) * E, E, row);
+    float v0 = -INFINITY, v1 = -INFINITY;
+    int i0 = -1, i1 = -1;
+#pragma unroll
+    for (int i = 0; i < PL; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E && (i0 < 0 || row.v[i] > v0)) {
+        v0 = row.v[i];
+        i0 = e;
+      }
+    }
+    warp_argmax(v0, i0);
+#pragma unroll
+    for (int i = 0; i < PL; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E && e != i0 && (i1 < 0 || row.v[i] > v1)) {
+        v1 = row.v[i];
+        i1 = e;
+      }
+    }
+    warp_argmax(v1, i1);
+    if (lane == 0) {
+      int b = 0;
+      if (!isinf(w)) {
+        if (i1 < 0) {
+          b = B - 1;
+        } else {
+          const double qd = static_cast<double>(v0 - v1) / w;
+          b = qd >= static_cast<double>(B - 1) ? B - 1 : static_cast<int>(floor(qd));
+        }
+      }
+      bin_s[t] = static_cast<uint8_t>(b);
+      if (bins_out) bins_out[t] = b;
+    }
+  }
+  for (int t = tid; t < T; t += blockDim.x) r0[idx_s[t * k]] = 1;
+  __syncthreads();
+  // S_e: one thread per expert scans the batch in (token, slot) order
+  for (int e = tid; e < E; e += blockDim.x) {
+    double sc = 0.0;
+    for (int t = 0, a = 0; t < T; ++t) {
+      const double wt = ldexp(1.0, bin_s[t]);
+      for (int s = 0; s < k; ++s, ++a)
+        if (idx_s[a] == e) sc += wt * static_cast<double>(gate[a]);
+    }
+    S[e] = sc;
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x)
+    if (r0[e]) atomicAdd(&n_r0, 1);
+  __syncthreads();
+  const int need = max(critical_n - n_r0, 0);
+  for (int e = tid; e < E; e += blockDim.x) {
+    bool c = r0[e];
+    if (!c) {
+      int rank = 0;
+      const double se = S[e];
+      for (int f = 0; f < E; ++f)
+        if (!r0[f] && (S[f] > se || (S[f] == se && f < e))) ++rank;
+      c = rank < need;
+    }
+    crit[e] = c ? 1 : 0;
+  }
+  __syncthreads();
+  if (critical)
+    for (int e = tid; e < E; e += blockDim.x) critical[e] = crit[e];
+  uint32_t crit_bits = 0;
+#pragma unroll
+  for (int i = 0; i < PL; ++i) {
+    const int e = lane + 32 * i;
+    if (e < E && crit[e]) crit_bits |= 1u << i;
+  }
+  for (int t = warp; t < T; t += nw) {
+    if (bin_s[t] >= low) continue;  // high-affinity token: its experts stay
     int cur[PW_MAX_TOPK];
     for (int j = 0; j < k; ++j) cur[j] = idx[static_cast<size_t>(t) * k + j];
     WarpRow<PL> row;

@@ -92,4 +92,45 @@ pw_status pw_remap(const float* logits, int32_t* idx, const float* gate, int T, 
   return launch_status();
 }
 
+pw_status pw_affinity_default(int E, int k, pw_affinity_cfg* out) {
+  if (!out || E < 1 || k < 1 || k > E) return PW_ERR_INVALID_ARG;
+  const double ratio = static_cast<double>(E) / k;
+  if (ratio <= 1.0) {
+    out->num_bins = 1;
+    out->low_bins = 1;
+    out->bin_width = INFINITY;
+    return PW_OK;
+  }
+  const int B = static_cast<int>(std::ceil(ratio));
+  out->num_bins = B;
+  out->low_bins = (B + 1) / 2;
+  out->bin_width = std::log(ratio) / B;
+  return PW_OK;
+}
+
+pw_status pw_affinity_remap(const float* logits, int32_t* idx, const float* gate, int T, int E,
+                            const pw_route_cfg* cfg, const pw_affinity_cfg* acfg,
+                            uint8_t* critical, int32_t* bins, pw_stream_t stream) {
+  if (!logits || !idx || !gate || !acfg) return PW_ERR_INVALID_ARG;
+  if (T < 1 || T > PW_MAX_TOKENS || E < 1 || E > PW_MAX_EXPERTS || !cfg_ok(cfg, E))
+    return PW_ERR_INVALID_ARG;
+  if (cfg->critical_n < 0 || static_cast<long long>(T) * cfg->k > 8192) return PW_ERR_INVALID_ARG;
+  const double w = acfg->bin_width;
+  if (acfg->num_bins < 1 || acfg->num_bins > 256 || acfg->low_bins < 0 || !(w > 0.0))
+    return PW_ERR_INVALID_ARG;  // also rejects a NaN width
+  cudaStream_t st = as_cuda(stream);
+#define PW_AFF(PL)                                                                            \
+  pw::affinity_remap_kernel<PL><<<1, 1024, 0, st>>>(logits, idx, gate, T, E, cfg->k,          \
+                                                    cfg->critical_n, acfg->num_bins, w,        \
+                                                    acfg->low_bins, critical, bins)
+  if (E <= 32) PW_AFF(1);
+  else if (E <= 64) PW_AFF(2);
+  else if (E <= 128) PW_AFF(4);
+  else if (E <= 256) PW_AFF(8);
+  else if (E <= 512) PW_AFF(16);
+  else PW_AFF(32);
+#undef PW_AFF
+  return launch_status();
+}
+
 }  // extern "C"

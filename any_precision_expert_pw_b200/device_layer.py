@@ -12,7 +12,8 @@ from typing import Optional
 import numpy as np
 
 from . import binding as B
-from .inputs import MIN_BITS, MOD_DOWN, MOD_GATE_UP, POLICY_NONE, POLICY_REMAP, SynthLayer
+from .inputs import (MIN_BITS, MOD_DOWN, MOD_GATE_UP, POLICY_AFFINITY, POLICY_NONE, POLICY_REMAP,
+                     SynthLayer)
 
 
 def _torch():
@@ -104,7 +105,14 @@ class DeviceLayer:
                                 self.idx.data_ptr(), self.gate.data_ptr(), self.stream),
                 "pw_route_topk")
         pol = self.cfg.policy
-        if pol == POLICY_REMAP:
+        if pol == POLICY_AFFINITY:
+            acfg = B.pw_affinity_cfg()
+            B.check(B.pw_affinity_default(self.E, self.k, acfg), "pw_affinity_default")
+            B.check(B.pw_affinity_remap(self.logits.data_ptr(), self.idx.data_ptr(),
+                                        self.gate.data_ptr(), self.T, self.E, self.route_cfg,
+                                        acfg, self.critical.data_ptr(), 0, self.stream),
+                    "pw_affinity_remap")
+        elif pol == POLICY_REMAP:
             B.check(B.pw_remap(self.logits.data_ptr(), self.idx.data_ptr(), self.gate.data_ptr(),
                                self.T, self.E, self.route_cfg, self.critical.data_ptr(),
                                self.stream), "pw_remap")

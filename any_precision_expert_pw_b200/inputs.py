@@ -46,6 +46,7 @@ POLICY_FETCH_ALL = 0
 POLICY_THRESHOLD = 1
 POLICY_FIRST_CHOICE = 2
 POLICY_REMAP = 3
+POLICY_AFFINITY = 4   # LYNX AffinityBinning remap (bins from k/N), in place of POLICY_REMAP
 
 
 @dataclasses.dataclass(frozen=True)

@@ -44,6 +44,9 @@ def parse_args():
     ap.add_argument("--impl", choices=("pw", "reference"), default="pw")
     ap.add_argument("--workload", default=f"{WORKLOAD[0]}:{WORKLOAD[1]}",
                     help="config name:T (default mixtral_8x7b:1)")
+    ap.add_argument("--affinity", action="store_true",
+                    help="rewrite the assignments with LYNX AffinityBinning (pw_affinity_remap) "
+                         "in place of the config's own rewrite")
     ap.add_argument("--skip-cpu-baseline", action="store_true",
                     help="leave out the CPU oracle timing (profiling runs)")
     ap.add_argument("--cpu-sample-rows", type=float, default=None,
@@ -52,9 +55,13 @@ def parse_args():
 
 
 def workload(args):
-    from any_precision_expert_pw_b200.inputs import CONFIGS
+    import dataclasses
+    from any_precision_expert_pw_b200.inputs import CONFIGS, POLICY_AFFINITY
     name, T = args.workload.split(":")
-    return CONFIGS[name], int(T)
+    cfg = CONFIGS[name]
+    if getattr(args, "affinity", False):
+        cfg = dataclasses.replace(cfg, policy=POLICY_AFFINITY)
+    return cfg, int(T)
 
 
 def read_peaks():
@@ -406,6 +413,8 @@ def run_pw(args):
         "config": {"workload": f"{cfg.name}-shaped MoE decode layer, T={T}", "H": cfg.H,
                    "E": cfg.E, "I": cfg.I, "k": cfg.k, "parent_bits": cfg.n,
                    "bits": L.q.tolist(), "experts_used": used.tolist(),
+                   "rewrite": {-1: "none", 0: "fetch-all", 1: "0.15 rule", 2: "first choice",
+                               3: "batch remap", 4: "AffinityBinning remap"}[cfg.policy],
                    "parallelism": f"replicas{world}" if world > 1 else "single",
                    "l2": "flushed before every step (memset of 2.5x L2, outside the step events)",
                    "timing": "CUDA-graph replay per step, CUDA events on the launching stream"},

@@ -204,6 +204,37 @@ pw_status pw_substitute(const float* logits, int32_t* idx, const float* gate,
 pw_status pw_remap(const float* logits, int32_t* idx, const float* gate, int T, int E,
                    const pw_route_cfg* cfg, uint8_t* critical, pw_stream_t stream);
 
+/* AffinityBinning configuration (pw_affinity_remap). */
+typedef struct pw_affinity_cfg {
+  int32_t num_bins;  /* B >= 1 (<= 256)                                                   */
+  int32_t low_bins;  /* tokens whose bin is < low_bins are low-affinity (remapped)          */
+  double bin_width;  /* w > 0, +inf allowed (every token in bin 0)                          */
+} pw_affinity_cfg;
+
+/* ---------------------------------------------------------------------------------------
+ * pw_affinity_default [LX2] (host only): the bins from the sparsity ratio k/N alone:
+ * B = ceil(E/k), w = ln(E/k) / B, low_bins = ceil(B/2); E/k <= 1 gives one bin of width +inf.
+ * ------------------------------------------------------------------------------------- */
+pw_status pw_affinity_default(int E, int k, pw_affinity_cfg* out);
+
+/* ---------------------------------------------------------------------------------------
+ * pw_affinity_remap [LX1][LX2]: LYNX AffinityBinning, in place.  The pages give the
+ * structure (confidence from the gap between the top-ranked logits, binned with widths set by
+ * k/N; batch expert scores with exponential weights of the bins; a critical set; low-affinity
+ * assignments remapped, k experts kept) but no formula; this is one reading of it:
+ *   d_t = fp32 gap between token t's two largest logits (ties: lower index ranks first);
+ *   bin_t = min(floor(d_t / w), B - 1) in float64 (B - 1 when E = 1, 0 when w = +inf);
+ *   S_e = sum over assignments (t, s) with idx = e of 2^bin_t * gate[t][s], float64 in
+ *         ascending (token, slot) order;
+ *   critical set C and the remap as in pw_remap with S_e in place of the gate sums, applied
+ *   only to tokens with bin_t < low_bins.  With w = +inf this is exactly pw_remap.
+ *   logits [T][E] fp32, idx [T][k] int32 (in/out), gate [T][k] fp32, critical [E] uint8 and
+ *   bins [T] int32 outputs (either may be NULL).  One thread block: T * k <= 8192.
+ * ------------------------------------------------------------------------------------- */
+pw_status pw_affinity_remap(const float* logits, int32_t* idx, const float* gate, int T, int E,
+                            const pw_route_cfg* cfg, const pw_affinity_cfg* acfg,
+                            uint8_t* critical, int32_t* bins, pw_stream_t stream);
+
 /* ---------------------------------------------------------------------------------------
  * pw_moe_workspace_bytes: device workspace needed by pw_moe_anyprec_forward (0 on bad args).
  * ------------------------------------------------------------------------------------- */

@@ -18,6 +18,8 @@ Sources (page title and section; the pages are summaries in French):
 * LYNX, 2.1 "Principes Fondamentaux" (rank-0 dominates) and 2.2 "Composants du Système"
   (batch-wide expert scores, a critical expert set, remapping that keeps exactly k experts).
 * LYNX, 1 "Énoncé du Problème" -- each token independently picks its top-k experts.
+* LYNX, 2.2 "Composants du Système" (Confidence Analyzer, Adaptive Expert Scorer) and 3 item 2
+  -- AffinityBinning (affinity.py).
 
 Everything the pages leave open is read the plainest way and stated where it is used: the
 plane layout (plane 0 = most significant bit, bit j of word w = column 32w+j), child index =
@@ -32,6 +34,10 @@ two-expert softmax), special cases (q = n equals the dense LUT-dequantised matri
 integer-valued LUTs that expose the decoded indices, all-resident = identity, +inf threshold =
 first-choice rule, critical set covering every chosen expert = identity), and invariants
 (exactly k distinct experts per token, top-1 never substituted, rank-0 never remapped).
-No function here is "parity unpinned".
+
+Parity unpinned: affinity.py (AffinityBinning).  The pages name its parts but give no formula,
+so what it computes is this project's reading (stated in its docstring); it is pinned against
+hand cases, a brute-force bin definition and the batch remap it reduces to, not against the
+pages.  Every other function is pinned as above.
 """
-from . import bitplanes, router, policy, group, ffn, layer  # noqa: F401
+from . import affinity, bitplanes, router, policy, group, ffn, layer  # noqa: F401

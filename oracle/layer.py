@@ -1,17 +1,20 @@
 """The whole decode layer, step by step (oracle; test infrastructure only).
 
-router GEMV -> softmax top-k -> (substitution | remap | nothing) -> grouped any-precision FFN ->
+router GEMV -> softmax top-k -> (substitution | remap | AffinityBinning remap | nothing) ->
+grouped any-precision FFN ->
 gate-weighted combine, as described in the module docstrings of router, policy, group and ffn.
 """
 from __future__ import annotations
 
 import numpy as np
 
+from . import affinity
 from . import policy as pol
 from .ffn import moe_ffn
 from .router import router_logits, softmax_topk
 
 POLICY_REMAP = 3
+POLICY_AFFINITY = 4
 
 
 def route(layer):
@@ -27,6 +30,11 @@ def route(layer):
     elif cfg.policy == POLICY_REMAP:
         idx2, crit = pol.remap(logits, idx, gate, cfg.critical_n)
         res.update(idx=idx2, critical=crit)
+    elif cfg.policy == POLICY_AFFINITY:
+        nb, w, low = affinity.default_bins(cfg.E, cfg.k)
+        idx2, crit, bins, _ = affinity.affinity_remap(logits, idx, gate, cfg.critical_n, nb, w,
+                                                      low)
+        res.update(idx=idx2, critical=crit, bins=bins)
     return res
 
 

@@ -62,6 +62,24 @@ def test_host_argument_checks(libpw):
     assert B.pw_commit_bits(0, 16, 16, 16, 1) == bad
 
 
+def test_affinity_defaults_and_argument_checks(libpw):
+    import math
+    from oracle.affinity import default_bins
+    for E, k in ((64, 8), (8, 2), (512, 10), (60, 4), (4, 4), (1, 1)):
+        a = B.pw_affinity_cfg()
+        assert B.pw_affinity_default(E, k, a) == B.PW_OK
+        nb, w, low = default_bins(E, k)
+        assert (a.num_bins, a.low_bins) == (nb, low)
+        assert (math.isinf(a.bin_width) and math.isinf(w)) or a.bin_width == w
+    bad = B.PW_ERR_INVALID_ARG
+    assert B.pw_affinity_default(8, 9, B.pw_affinity_cfg()) == bad
+    cfg = B.pw_route_cfg(k=2, renorm=1, policy=1, threshold=0.15, critical_n=4)
+    for a in (B.pw_affinity_cfg(0, 1, 0.5), B.pw_affinity_cfg(4, 2, 0.0),
+              B.pw_affinity_cfg(4, 2, float("nan")), B.pw_affinity_cfg(4, -1, 0.5)):
+        assert B.pw_affinity_remap(16, 16, 16, 4, 8, cfg, a, 0, 0, 0) == bad
+    assert B.pw_affinity_remap(16, 16, 16, 4, 8, cfg, None, 0, 0, 0) == bad
+
+
 def test_block_prepare_rejects_bad_blocks(libpw):
     blk = B.pw_block()
     assert B.pw_block_prepare(blk) == B.PW_ERR_INVALID_ARG                 # no planes
