@@ -36,7 +36,8 @@ PW_MAX_TOKENS = 4096
 
 # every symbol include/pw.h declares
 EXPORTS = ("pw_block_prepare", "pw_pack_bitplanes", "pw_route_topk", "pw_substitute",
-           "pw_remap", "pw_affinity_default", "pw_affinity_remap", "pw_moe_workspace_bytes",
+           "pw_remap", "pw_affinity_default", "pw_affinity_remap", "pw_cache_step",
+           "pw_moe_workspace_bytes",
            "pw_moe_anyprec_forward",
            "pw_moe_anyprec_forward_static", "pw_commit_bits", "pw_get_status",
            "pw_status_string", "pw_version")
@@ -96,6 +97,8 @@ def lib() -> ctypes.CDLL:
         L.pw_substitute.argtypes = [P, P, P, P, I, I, ctypes.POINTER(pw_route_cfg), P, P, S]
         L.pw_remap.argtypes = [P, P, P, I, I, ctypes.POINTER(pw_route_cfg), P, S]
         L.pw_affinity_default.argtypes = [I, I, ctypes.POINTER(pw_affinity_cfg)]
+        L.pw_cache_step.argtypes = [P, P, P, I, I, ctypes.POINTER(pw_route_cfg), ctypes.c_double,
+                                    P, P, P, I, P, P, P, S]
         L.pw_affinity_remap.argtypes = [P, P, P, I, I, ctypes.POINTER(pw_route_cfg),
                                         ctypes.POINTER(pw_affinity_cfg), P, P, S]
         L.pw_moe_workspace_bytes.argtypes = [I, I, I, I, I]
@@ -166,6 +169,12 @@ def pw_affinity_default(E, k, out) -> int:
 def pw_affinity_remap(logits, idx, gate, T, E, cfg, acfg, critical, bins, stream=0) -> int:
     return lib().pw_affinity_remap(logits, idx, gate, T, E, _cfg(cfg), _cfg(acfg), critical,
                                    bins, stream)
+
+
+def pw_cache_step(logits, idx, gate, T, E, cfg, beta, resident, mass, freq, capacity, action,
+                  mass_t, stats, stream=0) -> int:
+    return lib().pw_cache_step(logits, idx, gate, T, E, _cfg(cfg), float(beta), resident, mass,
+                               freq, capacity, action, mass_t, stats, stream)
 
 
 def pw_moe_workspace_bytes(T, k, E, H, I) -> int:

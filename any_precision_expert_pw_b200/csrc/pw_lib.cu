@@ -10,6 +10,7 @@
 #include <mutex>
 
 #include "pw.h"
+#include "pw_cache.cuh"
 #include "pw_common.cuh"
 #include "pw_ffn.cuh"
 #include "pw_group.cuh"

@@ -133,4 +133,34 @@ pw_status pw_affinity_remap(const float* logits, int32_t* idx, const float* gate
   return launch_status();
 }
 
+pw_status pw_cache_step(const float* logits, int32_t* idx, const float* gate, int T, int E,
+                        const pw_route_cfg* cfg, double beta, uint8_t* resident, double* mass,
+                        uint32_t* freq, int capacity, uint8_t* action, float* mass_t,
+                        int32_t* stats, pw_stream_t stream) {
+  if (!logits || !idx || !gate || !resident || !mass || !freq) return PW_ERR_INVALID_ARG;
+  if (T < 1 || T > PW_MAX_TOKENS || E < 1 || E > PW_MAX_EXPERTS || !cfg_ok(cfg, E))
+    return PW_ERR_INVALID_ARG;
+  if (static_cast<long long>(T) * cfg->k > pw::kCacheMaxAssign) return PW_ERR_INVALID_ARG;
+  if (cfg->policy != PW_POLICY_FETCH_ALL && cfg->policy != PW_POLICY_THRESHOLD &&
+      cfg->policy != PW_POLICY_FIRST_CHOICE)
+    return PW_ERR_INVALID_ARG;
+  if (cfg->threshold != cfg->threshold || beta != beta || capacity < 0 || capacity > E)
+    return PW_ERR_INVALID_ARG;
+  cudaStream_t st = as_cuda(stream);
+  if (stats && cudaMemsetAsync(stats, 0, 3 * sizeof(int32_t), st) != cudaSuccess)
+    return PW_ERR_CUDA;
+#define PW_CACHE(PL)                                                                          \
+  pw::cache_step_kernel<PL><<<1, 1024, 0, st>>>(logits, idx, gate, T, E, cfg->k, cfg->policy,  \
+                                                cfg->threshold, beta, resident, mass, freq,    \
+                                                capacity, action, mass_t, stats)
+  if (E <= 32) PW_CACHE(1);
+  else if (E <= 64) PW_CACHE(2);
+  else if (E <= 128) PW_CACHE(4);
+  else if (E <= 256) PW_CACHE(8);
+  else if (E <= 512) PW_CACHE(16);
+  else PW_CACHE(32);
+#undef PW_CACHE
+  return launch_status();
+}
+
 }  // extern "C"

@@ -216,3 +216,20 @@ def random_router_inputs(T: int, E: int, H: int, seed: int, zipf_s: Optional[flo
 def random_indices(R: int, C: int, n: int, seed: int) -> np.ndarray:
     rng = np.random.default_rng(np.random.SeedSequence([9002, R, C, n, seed]))
     return rng.integers(0, 1 << n, size=(R, C), dtype=np.uint8)
+
+
+def logit_stream(E: int, T: int, steps: int, seed: int, topic_len: int = 16,
+                 topic_scale: float = 2.0) -> np.ndarray:
+    """Router logits for a run of decode steps [steps][T][E] (fp32): standard normal noise plus
+    a per-topic bias that changes every `topic_len` steps (a random permutation of a Zipf(1.2)
+    log-profile times `topic_scale`), standing in for a real model's routing stream."""
+    rng = np.random.default_rng(np.random.SeedSequence([7, E, T, steps, seed]))
+    prof = np.log(np.arange(1, E + 1, dtype=np.float64) ** -1.2)
+    prof -= prof.mean()
+    out = np.empty((steps, T, E), dtype=np.float32)
+    bias = None
+    for s in range(steps):
+        if s % topic_len == 0:
+            bias = topic_scale * prof[rng.permutation(E)] / max(prof.std(), 1e-12)
+        out[s] = (rng.standard_normal((T, E)) + bias).astype(np.float32)
+    return out

@@ -236,6 +236,30 @@ pw_status pw_affinity_remap(const float* logits, int32_t* idx, const float* gate
                             uint8_t* critical, int32_t* bins, pw_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------
+ * pw_cache_step [SUB]: one decode step of an expert cache (Quality-First = PW_POLICY_THRESHOLD
+ * with threshold 0.15, Speed-First = PW_POLICY_FIRST_CHOICE; both with frequency-based
+ * eviction and background admission at beta = 0.5).  The pages list the components, not
+ * their order; this call does, on device state the caller owns:
+ *   1. freq[e] += 1 for every routed assignment (idx as given);
+ *   2. idx is rewritten in place by the rule of pw_substitute against resident[] as it is at
+ *      the start of the step (action, mass_t as in pw_substitute; either may be NULL);
+ *   3. mass[e] += gate of every substituted slot, e = the expert it replaced (float64,
+ *      ascending (token, slot) order);
+ *   4. inserted: the experts fetched this step (first occurrence order), then every other
+ *      non-resident expert with mass[e] >= beta; an inserted expert's mass becomes 0; if the
+ *      insertions alone exceed `capacity`, the most selected fetches and then the heaviest
+ *      admissions are kept (ties: lower index);
+ *   5. evicted: start-of-step residents, ordered by (used after the rewrite, freq, index),
+ *      until at most `capacity` experts are resident.
+ *   resident [E] uint8, mass [E] double, freq [E] uint32: in/out.  stats [3] int32 (may be
+ *   NULL): fetched, admitted, evicted.  One thread block: T * k <= 8192.
+ * ------------------------------------------------------------------------------------- */
+pw_status pw_cache_step(const float* logits, int32_t* idx, const float* gate, int T, int E,
+                        const pw_route_cfg* cfg, double beta, uint8_t* resident, double* mass,
+                        uint32_t* freq, int capacity, uint8_t* action, float* mass_t,
+                        int32_t* stats, pw_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
  * pw_moe_workspace_bytes: device workspace needed by pw_moe_anyprec_forward (0 on bad args).
  * ------------------------------------------------------------------------------------- */
 size_t pw_moe_workspace_bytes(int T, int k, int E, int H, int I);
