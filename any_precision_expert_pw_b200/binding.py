@@ -35,7 +35,7 @@ PW_MAX_TOPK = 16
 PW_MAX_TOKENS = 4096
 
 # every symbol include/pw.h declares
-EXPORTS = ("pw_block_prepare", "pw_pack_bitplanes", "pw_route_topk", "pw_substitute",
+EXPORTS = ("pw_block_prepare", "pw_pack_bitplanes", "pw_route_topk", "pw_topk", "pw_substitute",
            "pw_remap", "pw_affinity_default", "pw_affinity_remap", "pw_cache_step",
            "pw_moe_workspace_bytes",
            "pw_moe_anyprec_forward",
@@ -94,6 +94,7 @@ def lib() -> ctypes.CDLL:
         L.pw_block_prepare.argtypes = [ctypes.POINTER(pw_block)]
         L.pw_pack_bitplanes.argtypes = [P, I, I, I, I, P, S]
         L.pw_route_topk.argtypes = [P, P, P, I, I, I, ctypes.POINTER(pw_route_cfg), P, P, P, S]
+        L.pw_topk.argtypes = [P, I, I, ctypes.POINTER(pw_route_cfg), P, P, S]
         L.pw_substitute.argtypes = [P, P, P, P, I, I, ctypes.POINTER(pw_route_cfg), P, P, S]
         L.pw_remap.argtypes = [P, P, P, I, I, ctypes.POINTER(pw_route_cfg), P, S]
         L.pw_affinity_default.argtypes = [I, I, ctypes.POINTER(pw_affinity_cfg)]
@@ -152,6 +153,10 @@ def pw_pack_bitplanes(idx, rows, cols, n, layout, planes, stream=0) -> int:
 
 def pw_route_topk(x_bf16, Wr, bias, T, H, E, cfg, logits, idx, gate, stream=0) -> int:
     return lib().pw_route_topk(x_bf16, Wr, bias, T, H, E, _cfg(cfg), logits, idx, gate, stream)
+
+
+def pw_topk(logits, T, E, cfg, idx, gate, stream=0) -> int:
+    return lib().pw_topk(logits, T, E, _cfg(cfg), idx, gate, stream)
 
 
 def pw_substitute(logits, idx, gate, resident, T, E, cfg, action, mass, stream=0) -> int:

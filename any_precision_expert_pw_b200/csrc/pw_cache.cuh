@@ -1,14 +1,14 @@
 // Expert cache policy across decode steps ("Which Expert Misses Are Worth Waiting For?",
 // "Méthodologie" and "Contributions Clés" 5): the 0.15 / first-choice substitution against the
 // current resident set, frequency-based eviction and background admission of experts whose
-// accumulated substituted gate mass reaches beta.  One CTA per step (E <= 1024, T*k <= 8192).
+// accumulated substituted gate mass reaches beta.  One CTA per step (E <= 1024, T*k <= 4096).
 #pragma once
 #include "pw_common.cuh"
 #include "pw_route.cuh"
 
 namespace pw {
 
-constexpr int kCacheMaxAssign = 8192;
+constexpr int kCacheMaxAssign = 4096;
 
 template <int PL>
 __global__ void __launch_bounds__(1024) cache_step_kernel(
@@ -17,12 +17,14 @@ __global__ void __launch_bounds__(1024) cache_step_kernel(
     double* __restrict__ mass, uint32_t* __restrict__ freq, int capacity,
     uint8_t* __restrict__ action_out, float* __restrict__ mass_t, int32_t* __restrict__ stats) {
   __shared__ int16_t idx0_s[kCacheMaxAssign];  // the step's routed experts
+  __shared__ int16_t idx2_s[kCacheMaxAssign];  // after the rewrite
   __shared__ uint8_t act_s[kCacheMaxAssign];
   __shared__ double mass_s[PW_MAX_EXPERTS];
   __shared__ uint32_t freq_s[PW_MAX_EXPERTS];
   __shared__ uint8_t start[PW_MAX_EXPERTS];  // resident at the start of the step
   __shared__ uint8_t used[PW_MAX_EXPERTS];   // referenced after the rewrite
   __shared__ uint8_t ins[PW_MAX_EXPERTS];    // inserted this step
+  __shared__ uint8_t adm[PW_MAX_EXPERTS];    // background admission this step
   __shared__ int16_t flist[PW_MAX_EXPERTS], alist[PW_MAX_EXPERTS];
   __shared__ int bad, n_over, n_f, n_a, n_start;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
@@ -30,6 +32,8 @@ __global__ void __launch_bounds__(1024) cache_step_kernel(
   if (tid == 0) {
     bad = 0;
     n_start = 0;
+    n_f = 0;
+    n_a = 0;
   }
   for (int e = tid; e < E; e += blockDim.x) {
     start[e] = resident[e] ? 1 : 0;
@@ -37,6 +41,7 @@ __global__ void __launch_bounds__(1024) cache_step_kernel(
     freq_s[e] = freq[e];
     used[e] = 0;
     ins[e] = 0;
+    adm[e] = 0;
   }
   for (int a = tid; a < TK; a += blockDim.x) {
     const int e = idx[a];
@@ -91,6 +96,7 @@ __global__ void __launch_bounds__(1024) cache_step_kernel(
     if (lane == 0) {
       for (int s = 0; s < k; ++s) {
         idx[static_cast<size_t>(t) * k + s] = cur[s];
+        idx2_s[t * k + s] = static_cast<int16_t>(cur[s]);
         used[cur[s]] = 1;
         if (action_out) action_out[static_cast<size_t>(t) * k + s] = act_s[t * k + s];
       }
@@ -98,49 +104,64 @@ __global__ void __launch_bounds__(1024) cache_step_kernel(
     }
   }
   __syncthreads();
-  // 3. accumulated substituted mass (float64, ascending (token, slot)) and the insertions
-  if (tid == 0) {
+  // 3. accumulated substituted mass: one thread per expert adds its own substituted slots in
+  //    ascending (token, slot) order (float64); fetched experts are flagged by their slots
+  for (int e = tid; e < E; e += blockDim.x) {
+    double m = mass_s[e];
     for (int a = 0; a < TK; ++a)
-      if (act_s[a] == PW_ACT_SUBST) mass_s[idx0_s[a]] += static_cast<double>(gate[a]);
-    int nf = 0, na = 0;
-    for (int a = 0; a < TK; ++a) {
-      const int e = idx[a];
-      if (act_s[a] == PW_ACT_FETCH && !start[e] && !ins[e]) {
-        ins[e] = 1;
-        flist[nf++] = static_cast<int16_t>(e);
-      }
-    }
-    for (int e = 0; e < E; ++e)
-      if (!start[e] && !ins[e] && mass_s[e] >= beta) alist[na++] = static_cast<int16_t>(e);
-    if (nf + na > capacity) {  // keep the most selected fetches, then the heaviest admissions
-      for (int i = 0; i < nf; ++i)
-        for (int j = i + 1; j < nf; ++j) {
-          const int a = flist[i], b = flist[j];
-          if (freq_s[b] > freq_s[a] || (freq_s[b] == freq_s[a] && b < a)) {
-            flist[i] = static_cast<int16_t>(b);
-            flist[j] = static_cast<int16_t>(a);
-          }
-        }
-      for (int i = 0; i < na; ++i)
-        for (int j = i + 1; j < na; ++j) {
-          const int a = alist[i], b = alist[j];
-          if (mass_s[b] > mass_s[a] || (mass_s[b] == mass_s[a] && b < a)) {
-            alist[i] = static_cast<int16_t>(b);
-            alist[j] = static_cast<int16_t>(a);
-          }
-        }
-      for (int i = 0; i < nf; ++i) ins[flist[i]] = 0;
-      nf = min(nf, capacity);
-      na = min(na, max(capacity - nf, 0));
-      for (int i = 0; i < nf; ++i) ins[flist[i]] = 1;
-    }
-    for (int i = 0; i < na; ++i) ins[alist[i]] = 1;
-    for (int i = 0; i < nf; ++i) mass_s[flist[i]] = 0.0;
-    for (int i = 0; i < na; ++i) mass_s[alist[i]] = 0.0;
-    n_f = nf;
-    n_a = na;
-    n_over = n_start + nf + na - capacity;
+      if (idx0_s[a] == e && act_s[a] == PW_ACT_SUBST) m += static_cast<double>(gate[a]);
+    mass_s[e] = m;
   }
+  for (int a = tid; a < TK; a += blockDim.x) {
+    const int e = idx2_s[a];
+    if (act_s[a] == PW_ACT_FETCH && !start[e]) ins[e] = 1;  // every writer stores 1
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) {
+    if (ins[e]) atomicAdd(&n_f, 1);
+    else if (!start[e] && mass_s[e] >= beta) {
+      adm[e] = 1;
+      atomicAdd(&n_a, 1);
+    }
+  }
+  __syncthreads();
+  if (tid == 0 && n_f + n_a > capacity) {
+    // more insertions than the cache holds (rare): keep the most selected fetches, then the
+    // heaviest admissions (ties: lower index)
+    int nf = 0, na = 0;
+    for (int e = 0; e < E; ++e) {
+      if (ins[e]) flist[nf++] = static_cast<int16_t>(e);
+      if (adm[e]) alist[na++] = static_cast<int16_t>(e);
+    }
+    for (int i = 0; i < nf; ++i)
+      for (int j = i + 1; j < nf; ++j) {
+        const int a = flist[i], b = flist[j];
+        if (freq_s[b] > freq_s[a] || (freq_s[b] == freq_s[a] && b < a)) {
+          flist[i] = static_cast<int16_t>(b);
+          flist[j] = static_cast<int16_t>(a);
+        }
+      }
+    for (int i = 0; i < na; ++i)
+      for (int j = i + 1; j < na; ++j) {
+        const int a = alist[i], b = alist[j];
+        if (mass_s[b] > mass_s[a] || (mass_s[b] == mass_s[a] && b < a)) {
+          alist[i] = static_cast<int16_t>(b);
+          alist[j] = static_cast<int16_t>(a);
+        }
+      }
+    const int kf = min(nf, capacity), ka = min(na, max(capacity - kf, 0));
+    for (int i = kf; i < nf; ++i) ins[flist[i]] = 0;
+    for (int i = ka; i < na; ++i) adm[alist[i]] = 0;
+    n_f = kf;
+    n_a = ka;
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x)
+    if (ins[e] || adm[e]) {
+      ins[e] = 1;
+      mass_s[e] = 0.0;
+    }
+  if (tid == 0) n_over = n_start + n_f + n_a - capacity;
   __syncthreads();
   // 4. evictions: start residents ranked by (used, selections, index), the first n_over go
   int n_ev = 0;

@@ -37,14 +37,7 @@ pw_status pw_route_topk(const uint16_t* x_bf16, const float* Wr, const float* bi
   }
   if (launch_status() != PW_OK) return PW_ERR_CUDA;
   if (fuse_k) return PW_OK;
-  const int tg = (T + 7) / 8;
-  if (E <= 32) pw::topk_kernel<1><<<tg, 256, 0, st>>>(logits, T, E, cfg->k, cfg->renorm, idx, gate);
-  else if (E <= 64) pw::topk_kernel<2><<<tg, 256, 0, st>>>(logits, T, E, cfg->k, cfg->renorm, idx, gate);
-  else if (E <= 128) pw::topk_kernel<4><<<tg, 256, 0, st>>>(logits, T, E, cfg->k, cfg->renorm, idx, gate);
-  else if (E <= 256) pw::topk_kernel<8><<<tg, 256, 0, st>>>(logits, T, E, cfg->k, cfg->renorm, idx, gate);
-  else if (E <= 512) pw::topk_kernel<16><<<tg, 256, 0, st>>>(logits, T, E, cfg->k, cfg->renorm, idx, gate);
-  else pw::topk_kernel<32><<<tg, 256, 0, st>>>(logits, T, E, cfg->k, cfg->renorm, idx, gate);
-  return launch_status();
+  return pw_topk(logits, T, E, cfg, idx, gate, stream);
 }
 
 pw_status pw_substitute(const float* logits, int32_t* idx, const float* gate,
@@ -89,6 +82,25 @@ pw_status pw_remap(const float* logits, int32_t* idx, const float* gate, int T, 
   else if (E <= 512) PW_REMAP(16);
   else PW_REMAP(32);
 #undef PW_REMAP
+  return launch_status();
+}
+
+pw_status pw_topk(const float* logits, int T, int E, const pw_route_cfg* cfg, int32_t* idx,
+                  float* gate, pw_stream_t stream) {
+  if (!logits || !idx || !gate) return PW_ERR_INVALID_ARG;
+  if (T < 1 || T > PW_MAX_TOKENS || E < 1 || E > PW_MAX_EXPERTS || !cfg_ok(cfg, E))
+    return PW_ERR_INVALID_ARG;
+  const int tg = (T + 7) / 8;
+  cudaStream_t st = as_cuda(stream);
+#define PW_TOPK(PL)                                                                           \
+  pw::topk_kernel<PL><<<tg, 256, 0, st>>>(logits, T, E, cfg->k, cfg->renorm, idx, gate)
+  if (E <= 32) PW_TOPK(1);
+  else if (E <= 64) PW_TOPK(2);
+  else if (E <= 128) PW_TOPK(4);
+  else if (E <= 256) PW_TOPK(8);
+  else if (E <= 512) PW_TOPK(16);
+  else PW_TOPK(32);
+#undef PW_TOPK
   return launch_status();
 }
 

@@ -47,6 +47,9 @@ def parse_args():
     ap.add_argument("--affinity", action="store_true",
                     help="rewrite the assignments with LYNX AffinityBinning (pw_affinity_remap) "
                          "in place of the config's own rewrite")
+    ap.add_argument("--cache-stream", choices=("quality", "speed", "fetch-all"), default=None,
+                    help="instead of the layer step: drive pw_topk + pw_cache_step over a "
+                         "synthetic multi-step logit stream of the workload's router shape")
     ap.add_argument("--skip-cpu-baseline", action="store_true",
                     help="leave out the CPU oracle timing (profiling runs)")
     ap.add_argument("--cpu-sample-rows", type=float, default=None,
@@ -446,8 +449,91 @@ def run_pw(args):
     rep.close()
 
 
+def run_cache_stream(args):
+    """Expert cache across decode steps: one step = pw_topk + pw_cache_step on the next logits
+    of a seeded stream (topic changes every 32 steps); device time per step from CUDA events,
+    and what the policy did per token (fetches, admissions, evictions, substitutions)."""
+    import numpy as np
+    import torch
+
+    from any_precision_expert_pw_b200 import binding as B
+    from any_precision_expert_pw_b200.inputs import logit_stream
+
+    rep = Replicas("nccl")
+    dev = torch.device(f"cuda:{rep.local}")
+    torch.cuda.set_device(dev)
+    cfg, T = workload(args)
+    E, k = cfg.E, cfg.k
+    policy = {"quality": 1, "speed": 2, "fetch-all": 0}[args.cache_stream]
+    frac = cfg.resident_frac if cfg.resident_frac else 0.25
+    cap = int(frac * E)
+    steps, warm = args.steps, args.warmup
+    lo = torch.from_numpy(logit_stream(E, T, warm + steps, seed=1 + rep.rank, topic_len=32)).to(dev)
+    res0 = np.zeros(E, np.uint8)
+    res0[np.random.default_rng(np.random.SeedSequence([11, E, rep.rank])).choice(
+        E, cap, replace=False)] = 1
+    d_res = torch.from_numpy(res0).to(dev)
+    d_mass = torch.zeros(E, dtype=torch.float64, device=dev)
+    d_freq = torch.zeros(E, dtype=torch.int32, device=dev)
+    d_idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    d_gate = torch.empty((T, k), dtype=torch.float32, device=dev)
+    d_act = torch.empty((warm + steps, T, k), dtype=torch.uint8, device=dev)
+    d_m = torch.empty((warm + steps, T), dtype=torch.float32, device=dev)
+    d_stats = torch.zeros((warm + steps, 3), dtype=torch.int32, device=dev)
+    rcfg = B.pw_route_cfg(k=k, renorm=int(cfg.renorm), policy=policy, threshold=0.15,
+                          critical_n=0)
+    stream = torch.cuda.Stream(device=dev)
+    cs = stream.cuda_stream
+    evs = []
+    rep.barrier()
+    with torch.cuda.stream(stream):
+        for s in range(warm + steps):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            B.check(B.pw_topk(lo[s].data_ptr(), T, E, rcfg, d_idx.data_ptr(), d_gate.data_ptr(),
+                              cs), "pw_topk")
+            B.check(B.pw_cache_step(lo[s].data_ptr(), d_idx.data_ptr(), d_gate.data_ptr(), T, E,
+                                    rcfg, 0.5, d_res.data_ptr(), d_mass.data_ptr(),
+                                    d_freq.data_ptr(), cap, d_act[s].data_ptr(),
+                                    d_m[s].data_ptr(), d_stats[s].data_ptr(), cs),
+                    "pw_cache_step")
+            e1.record(stream)
+            if s >= warm:
+                evs.append((e0, e1))
+    torch.cuda.synchronize(dev)
+    rep.barrier()
+    st = B.pw_get_status(cs)
+    if st != B.PW_OK:
+        raise RuntimeError(f"device status: {B.pw_status_string(st)}")
+    ms = rep.max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / len(evs))
+    stats = d_stats[warm:].sum(0).cpu().numpy()
+    tokens = steps * T
+    out = {"metric": "expert-cache decode step (pw_topk + pw_cache_step)",
+           "value": rep.world * 1e3 / ms, "unit": "steps/s", "n_gpus": rep.world,
+           "steps": steps, "warmup": warm, "ms_per_step": ms, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f32/f64", "data": "synthetic",
+           "config": {"workload": f"{cfg.name}-shaped router stream, T={T}",
+                      "policy": {1: "Quality-First (0.15 rule)", 2: "Speed-First (first choice)",
+                                 0: "fetch every miss"}[policy] +
+                      " + frequency eviction + background admission (beta 0.5)",
+                      "E": E, "k": k, "capacity": cap, "topic_len": 32},
+           "fetched_per_token": float(stats[0]) / tokens,
+           "admitted_per_token": float(stats[1]) / tokens,
+           "evicted_per_token": float(stats[2]) / tokens,
+           "substituted_per_token": float((d_act[warm:] == 2).sum().item()) / tokens,
+           "mean_substituted_mass": float(d_m[warm:].mean().item()),
+           "gpu_launches": 2 * steps}
+    if rep.rank == 0:
+        print(json.dumps(out), flush=True)
+    rep.close()
+
+
 def main():
     args = parse_args()
+    if args.cache_stream:
+        run_cache_stream(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -176,6 +176,13 @@ pw_status pw_route_topk(const uint16_t* x_bf16, const float* Wr, const float* bi
                         float* gate, pw_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------
+ * pw_topk [LX1]: the selection half of pw_route_topk on logits the caller already has:
+ * logits [T][E] fp32 -> idx [T][k] int32, gate [T][k] fp32, same rules.
+ * ------------------------------------------------------------------------------------- */
+pw_status pw_topk(const float* logits, int T, int E, const pw_route_cfg* cfg, int32_t* idx,
+                  float* gate, pw_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
  * pw_substitute [SUB]: residency-aware rewrite of the routed assignments, in place.
  * For each token, slots in rank order: a resident expert is a hit; a missing one is fetched
  * (kept, counted) when the policy says so (rank 0, or gate >= threshold for
@@ -252,7 +259,7 @@ pw_status pw_affinity_remap(const float* logits, int32_t* idx, const float* gate
  *   5. evicted: start-of-step residents, ordered by (used after the rewrite, freq, index),
  *      until at most `capacity` experts are resident.
  *   resident [E] uint8, mass [E] double, freq [E] uint32: in/out.  stats [3] int32 (may be
- *   NULL): fetched, admitted, evicted.  One thread block: T * k <= 8192.
+ *   NULL): fetched, admitted, evicted.  One thread block: T * k <= 4096.
  * ------------------------------------------------------------------------------------- */
 pw_status pw_cache_step(const float* logits, int32_t* idx, const float* gate, int T, int E,
                         const pw_route_cfg* cfg, double beta, uint8_t* resident, double* mass,

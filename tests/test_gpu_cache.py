@@ -79,3 +79,18 @@ def test_cache_all_resident_and_infinite_beta(torch_dev):
     assert t.tolist() == [0, 0, 0]
     t = _run(torch, 64, 8, 4, 10, 16, op.POLICY_FIRST_CHOICE, 0.15, float("inf"), seed=4)
     assert t[1] == 0
+
+
+@pytest.mark.parametrize("E,k,T,renorm", [(512, 10, 16, True), (64, 8, 33, False), (8, 2, 5, True)])
+def test_topk_from_logits(torch_dev, E, k, T, renorm):
+    torch, dev = torch_dev
+    lo = logit_stream(E, T, 1, seed=E + k, topic_len=1)[0]
+    d_lo = torch.from_numpy(lo).to(dev)
+    d_idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    d_g = torch.empty((T, k), dtype=torch.float32, device=dev)
+    cfg = B.pw_route_cfg(k=k, renorm=int(renorm), policy=0, threshold=0.15, critical_n=0)
+    cs = torch.cuda.current_stream().cuda_stream
+    B.check(B.pw_topk(d_lo.data_ptr(), T, E, cfg, d_idx.data_ptr(), d_g.data_ptr(), cs))
+    idx, g, _ = softmax_topk(lo, k, renorm)
+    assert np.array_equal(d_idx.cpu().numpy(), idx)
+    assert np.max(np.abs(d_g.cpu().numpy() - g)) <= 1e-6
