@@ -36,7 +36,8 @@ PW_MAX_TOKENS = 4096
 
 # every symbol include/pw.h declares
 EXPORTS = ("pw_block_prepare", "pw_pack_bitplanes", "pw_route_topk", "pw_topk", "pw_substitute",
-           "pw_remap", "pw_affinity_default", "pw_affinity_remap", "pw_cache_step",
+           "pw_remap", "pw_affinity_default", "pw_affinity_remap", "pw_cache_step", "pw_page_copy", "pw_page_update",
+           "pw_plan_bitwidths",
            "pw_moe_workspace_bytes",
            "pw_moe_anyprec_forward",
            "pw_moe_anyprec_forward_static", "pw_commit_bits", "pw_get_status",
@@ -55,7 +56,7 @@ class pw_block(ctypes.Structure):
                 ("parent_bits", ctypes.c_uint8), ("min_bits", ctypes.c_uint8),
                 ("desired_bits", ctypes.c_uint8), ("committed_bits", ctypes.c_uint8),
                 ("state", ctypes.c_uint8), ("layout", ctypes.c_uint8),
-                ("reserved0", ctypes.c_uint8 * 2),
+                ("stored_bits", ctypes.c_uint8), ("reserved0", ctypes.c_uint8 * 1),
                 ("planes", ctypes.c_void_p), ("lut", ctypes.c_void_p * 9),
                 ("reserved1", ctypes.c_uint8 * 160)]
 
@@ -107,6 +108,9 @@ def lib() -> ctypes.CDLL:
         L.pw_moe_anyprec_forward.argtypes = [P, I, I, P, I, I, I, I, P, P, P, P, Z, S]
         L.pw_moe_anyprec_forward_static.argtypes = [P, I, I, P, I, I, I, I, P, P, P, S]
         L.pw_commit_bits.argtypes = [P, I, P, P, I, S]
+        L.pw_page_copy.argtypes = [P, I, P, I, I, I, I, S]
+        L.pw_page_update.argtypes = [P, I, P, I, S]
+        L.pw_plan_bitwidths.argtypes = [I, P, P, P, P, ctypes.c_uint64, P]
         L.pw_get_status.argtypes = [S]
         L.pw_status_string.argtypes = [I]
         L.pw_status_string.restype = ctypes.c_char_p
@@ -202,6 +206,28 @@ def pw_moe_anyprec_forward_static(pt_dev, layer, E, x_bf16, T, H, I, k, idx, gat
 
 def pw_commit_bits(pt_dev, num_blocks, block_ids, q, count, stream=0) -> int:
     return lib().pw_commit_bits(pt_dev, num_blocks, block_ids, q, count, stream)
+
+
+def pw_page_copy(src, src_bits, dst, dst_bits, rows, cols, q, stream=0) -> int:
+    return lib().pw_page_copy(src, src_bits, dst, dst_bits, rows, cols, q, stream)
+
+
+def pw_page_update(pt_dev, num_blocks, updates, count, stream=0) -> int:
+    return lib().pw_page_update(pt_dev, num_blocks, updates, count, stream)
+
+
+def pw_plan_bitwidths(nblocks, damage, bytes_, qmin, qmax, budget, q_out) -> int:
+    """Host arrays as integer addresses (e.g. numpy arr.ctypes.data)."""
+    return lib().pw_plan_bitwidths(nblocks, damage, bytes_, qmin, qmax, int(budget), q_out)
+
+
+class pw_page_update_t(ctypes.Structure):
+    _fields_ = [("block", ctypes.c_int32), ("state", ctypes.c_uint8),
+                ("stored_bits", ctypes.c_uint8), ("committed_bits", ctypes.c_uint8),
+                ("reserved", ctypes.c_uint8), ("planes", ctypes.c_void_p)]
+
+
+assert ctypes.sizeof(pw_page_update_t) == 16
 
 
 def pw_get_status(stream=0) -> int:

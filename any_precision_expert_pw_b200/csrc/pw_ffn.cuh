@@ -152,9 +152,11 @@ __device__ __forceinline__ Item resolve(const Params& p, int item) {
   const int nst = (p.cols + kStageCols - 1) / kStageCols;
   it.s0 = (nst * it.ks) / p.kslices;
   it.s1 = (nst * (it.ks + 1)) / p.kslices;
-  const bool bits_ok = it.q >= b->min_bits && it.q <= b->parent_bits && it.q >= PW_MIN_BITS &&
+  // planes held per (tile, stage) run on the device: all parent_bits, or a paged-in prefix
+  it.n = b->stored_bits ? b->stored_bits : b->parent_bits;
+  const bool bits_ok = it.q >= b->min_bits && it.q <= it.n && it.n <= b->parent_bits &&
+                       it.q >= PW_MIN_BITS &&
                        it.q <= PW_MAX_BITS && b->lut[it.q] != nullptr && b->planes != nullptr;
-  it.n = b->parent_bits;
   it.planes = b->planes + static_cast<size_t>(it.tile) * it.n * kRows * (p.cols / 32);
   const int want_layout = p.mode == MODE_GATE_UP ? PW_LAYOUT_TILED_GATE_UP : PW_LAYOUT_TILED_DOWN;
   const bool shape_ok = static_cast<int>(b->rows) == p.rows &&

@@ -48,6 +48,7 @@ class DeviceLayer:
         self.num_blocks = 2 * cfg.E
         self.blocks_host = (B.pw_block * self.num_blocks)()
         self._keep = []
+        self.planes = {}  # (expert, module) -> device plane buffer (tiled, all n planes)
         for e in range(cfg.E):
             for m in (MOD_GATE_UP, MOD_DOWN):
                 R, C = L.block_shape(m)
@@ -73,6 +74,7 @@ class DeviceLayer:
                     off += R * (1 << b)
                 B.check(B.pw_block_prepare(blk), "pw_block_prepare")
                 self._keep += [planes, lut_d]
+                self.planes[(e, m)] = planes
         self.blocks_dev = _bytes_tensor(self.blocks_host, self.device)
         self.pt_host = B.pw_page_table(1, cfg.E, self.blocks_dev.data_ptr())
         self.pt_dev = _bytes_tensor(self.pt_host, self.device)
@@ -153,6 +155,22 @@ class DeviceLayer:
         """[E, 2] committed bitwidths as stored in the device page table."""
         raw = self.blocks_dev.view(-1, 256)[:, 11].cpu().numpy()
         return raw.reshape(self.E, 2)
+
+    def page_update(self, updates) -> None:
+        """Apply pw_page_update_t edits (a list of dicts: block, state, stored_bits,
+        committed_bits, planes) to the device table, stream-ordered."""
+        torch = _torch()
+        arr = (B.pw_page_update_t * len(updates))()
+        for i, u in enumerate(updates):
+            arr[i].block = u["block"]
+            arr[i].state = u.get("state", -1) + 1
+            arr[i].stored_bits = u.get("stored_bits", 0)
+            arr[i].committed_bits = u.get("committed_bits", 0)
+            arr[i].planes = u.get("planes", None)
+        d = _bytes_tensor(arr, self.device)
+        B.check(B.pw_page_update(self.pt_dev.data_ptr(), self.num_blocks, d.data_ptr(),
+                                 len(updates), self.stream), "pw_page_update")
+        self._keep.append(d)
 
     def set_state(self, e: int, m: int, state: int) -> None:
         """Change a block's page state in the device table (host-side test hook)."""

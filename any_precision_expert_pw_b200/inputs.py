@@ -233,3 +233,16 @@ def logit_stream(E: int, T: int, steps: int, seed: int, topic_len: int = 16,
             bias = topic_scale * prof[rng.permutation(E)] / max(prof.std(), 1e-12)
         out[s] = (rng.standard_normal((T, E)) + bias).astype(np.float32)
     return out
+
+
+def synthetic_damage(num_blocks: int, seed: int, hot_frac: float = 0.1,
+                     hot_mult: float = 4.0) -> np.ndarray:
+    """Per-block damage scores [num_blocks][9] (float64) for the bitwidth planner: a seeded
+    log-normal sensitivity per block, times a multiplier for a seeded set of hot blocks, times
+    4^-q (one more bit quarters the squared quantisation error); column q, q = 0..8."""
+    rng = np.random.default_rng(np.random.SeedSequence([13, num_blocks, seed]))
+    sens = rng.lognormal(mean=0.0, sigma=1.0, size=num_blocks)
+    hot = rng.random(num_blocks) < hot_frac
+    sens = sens * np.where(hot, hot_mult, 1.0)
+    q = np.arange(9, dtype=np.float64)
+    return sens[:, None] * np.power(4.0, -q)[None, :]

@@ -50,6 +50,9 @@ def parse_args():
     ap.add_argument("--cache-stream", choices=("quality", "speed", "fetch-all"), default=None,
                     help="instead of the layer step: drive pw_topk + pw_cache_step over a "
                          "synthetic multi-step logit stream of the workload's router shape")
+    ap.add_argument("--page-in", type=int, default=None, metavar="Q",
+                    help="instead of the layer step: page one expert of the workload in at "
+                         "bitwidth Q (top-Q planes of both blocks, pinned host -> device)")
     ap.add_argument("--skip-cpu-baseline", action="store_true",
                     help="leave out the CPU oracle timing (profiling runs)")
     ap.add_argument("--cpu-sample-rows", type=float, default=None,
@@ -529,8 +532,89 @@ def run_cache_stream(args):
     rep.close()
 
 
+def run_page_in(args):
+    """Page movement: one expert's two blocks move from pinned host memory (all n planes per
+    run) to compact device buffers holding the top q planes per run (pw_page_copy), then the
+    table entries are switched over (pw_page_update).  Device time per expert from CUDA events;
+    plane bytes moved per second."""
+    import numpy as np
+    import torch
+
+    from any_precision_expert_pw_b200 import binding as B
+    from any_precision_expert_pw_b200.device_layer import DeviceLayer
+    from any_precision_expert_pw_b200.inputs import MOD_DOWN, MOD_GATE_UP, make_layer
+
+    rep = Replicas("nccl")
+    dev = torch.device(f"cuda:{rep.local}")
+    torch.cuda.set_device(dev)
+    cfg, T = workload(args)
+    q = int(args.page_in)
+    n = cfg.n
+    if not (3 <= q <= n):
+        raise SystemExit(f"--page-in needs 3 <= Q <= {n}")
+    L = make_layer(cfg, T)
+    D = DeviceLayer(L, device=str(dev))
+    stream = torch.cuda.Stream(device=dev)
+    D.stream = stream.cuda_stream
+    e = 0
+    blocks = []
+    for m in (MOD_GATE_UP, MOD_DOWN):
+        R, C = L.block_shape(m)
+        host = torch.empty((n * R * C // 32,), dtype=torch.int32).pin_memory()
+        host.copy_(D.planes[(e, m)].cpu())
+        comp = torch.empty((q * R * C // 32,), dtype=torch.int32, device=dev)
+        blocks.append((m, R, C, host, comp))
+    moved = sum(q * R * C // 8 for _, R, C, _, _ in blocks)
+    ups = (B.pw_page_update_t * 2)()
+    for i, (m, R, C, host, comp) in enumerate(blocks):
+        ups[i].block = e * 2 + m
+        ups[i].state = B.PW_PAGE_GPU + 1
+        ups[i].stored_bits = q
+        ups[i].committed_bits = q
+        ups[i].planes = comp.data_ptr()
+    ups_d = torch.frombuffer(bytearray(bytes(ups)), dtype=torch.uint8).to(dev)
+    cs = stream.cuda_stream
+    evs = []
+    rep.barrier()
+    with torch.cuda.stream(stream):
+        for s in range(args.warmup + args.steps):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for m, R, C, host, comp in blocks:
+                B.check(B.pw_page_copy(host.data_ptr(), n, comp.data_ptr(), q, R, C, q, cs),
+                        "pw_page_copy")
+            B.check(B.pw_page_update(D.pt_dev.data_ptr(), D.num_blocks, ups_d.data_ptr(), 2, cs),
+                    "pw_page_update")
+            e1.record(stream)
+            if s >= args.warmup:
+                evs.append((e0, e1))
+    torch.cuda.synchronize(dev)
+    rep.barrier()
+    st = B.pw_get_status(cs)
+    if st != B.PW_OK:
+        raise RuntimeError(f"device status: {B.pw_status_string(st)}")
+    ms = rep.max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / len(evs))
+    full = sum(n * R * C // 8 for _, R, C, _, _ in blocks)
+    out = {"metric": "expert page-in (top-q planes, pinned host -> device)",
+           "value": rep.world * moved / (ms * 1e-3) / 1e9, "unit": "GB/s", "n_gpus": rep.world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u32",
+           "data": "synthetic",
+           "config": {"workload": f"{cfg.name}-shaped expert (gate_up + down), q={q} of n={n}",
+                      "bytes_moved": moved, "bytes_all_planes": full,
+                      "copies_per_step": sum((C // 32 + 31) // 32 for _, _, C, _, _ in blocks)},
+           "gpu_launches": args.steps}
+    if rep.rank == 0:
+        print(json.dumps(out), flush=True)
+    rep.close()
+
+
 def main():
     args = parse_args()
+    if args.page_in is not None:
+        run_page_in(args)
+        return
     if args.cache_stream:
         run_cache_stream(args)
         return

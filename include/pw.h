@@ -106,6 +106,9 @@ enum { PW_ACT_HIT = 0, PW_ACT_FETCH = 1, PW_ACT_SUBST = 2 };
  *     (n = parent_bits).  Reading the top q planes of (t, s) reads the first q * 32 * ws words
  *     of that run.  `layout` holds PW_LAYOUT_TILED_GATE_UP or PW_LAYOUT_TILED_DOWN; the
  *     forward checks it against the module.  `planes` is 16-byte aligned.
+ *   stored_bits: how many planes each (tile, stage) run holds in `planes` (0 = parent_bits):
+ *     a block paged in at bitwidth q (pw_page_copy) keeps only its top q planes on the device,
+ *     runs packed with that stride, so committed_bits may not exceed it.
  *   lut[b]: fp16 [rows][1<<b] for every b in [min_bits, parent_bits] (NULL otherwise);
  *           weight(r, c) at bitwidth q = lut[q][r][top q bits of idx(r, c)].
  *   committed_bits (q_i) is read once per forward call; desired_bits (d_i) is stored for a
@@ -122,7 +125,8 @@ typedef struct pw_block {
   uint8_t committed_bits;
   uint8_t state;
   uint8_t layout;
-  uint8_t reserved0[2];
+  uint8_t stored_bits;
+  uint8_t reserved0[1];
   const uint32_t* planes;
   const uint16_t* lut[9];
   uint8_t reserved1[160];
@@ -324,6 +328,52 @@ pw_status pw_moe_anyprec_forward_static(const pw_page_table* pt_dev, int layer, 
  * ------------------------------------------------------------------------------------- */
 pw_status pw_commit_bits(pw_page_table* pt_dev, int num_blocks, const int32_t* block_ids,
                          const uint8_t* q, int count, pw_stream_t stream);
+
+/* One page-table edit for pw_page_update: block id (layer*E + e)*2 + module; each other field
+ * 0 / NULL = leave unchanged.  state holds PW_PAGE_* + 1. */
+typedef struct pw_page_update_t {
+  int32_t block;
+  uint8_t state;          /* PW_PAGE_GPU + 1, PW_PAGE_CPU + 1, PW_PAGE_XFER + 1, or 0 */
+  uint8_t stored_bits;    /* planes per run now held by `planes` (min_bits..parent_bits) */
+  uint8_t committed_bits; /* q_i (min_bits..stored bits)                                 */
+  uint8_t reserved;
+  const uint32_t* planes; /* new device plane buffer (16-byte aligned), or NULL            */
+} pw_page_update_t;
+
+/* ---------------------------------------------------------------------------------------
+ * pw_page_copy [PW1][PW3]: page movement of Any-Precision planes.  Copies the top q planes of
+ * every (tile, stage) run between two buffers of the same block in the tiled layout holding
+ * src_bits and dst_bits planes per run (q <= both): host -> device (page in at bitwidth q,
+ * the device copy keeping only q planes per run), device -> host, device -> device.  Host
+ * buffers must be pinned for the copy to be asynchronous.  One pitched copy per 1024-column
+ * stage, on `stream`.  rows % 32 == 0, cols % 128 == 0, both pointers 16-byte aligned.
+ * ------------------------------------------------------------------------------------- */
+pw_status pw_page_copy(const uint32_t* src, int src_bits, uint32_t* dst, int dst_bits, int rows,
+                       int cols, int q, pw_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * pw_page_update [PW1][PW3]: applies `count` page-table edits (device array of
+ * pw_page_update_t) in stream order, e.g. state XFER before a pw_page_copy and
+ * {GPU, stored_bits = q, committed_bits = q, planes = new buffer} after it, so a forward
+ * ordered after the update sees a consistent entry, and one racing the transfer sees XFER
+ * (PW_ERR_NOT_RESIDENT, zeros).  Inconsistent edits are skipped with PW_ERR_BAD_BITS.
+ * ------------------------------------------------------------------------------------- */
+pw_status pw_page_update(pw_page_table* pt_dev, int num_blocks, const pw_page_update_t* updates,
+                         int count, pw_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------
+ * pw_plan_bitwidths [PW1] (host only): the damage-greedy bitwidth planner.  For nblocks
+ * blocks, damage[i][q] and bytes[i][q] (row-major [nblocks][PW_MAX_BITS + 1], read for q in
+ * [qmin[i], qmax[i]]): start every block at qmax, then, while the total bytes exceed `budget`,
+ * lower by one bit the block whose step adds the least damage per byte saved
+ * ((damage[i][q-1] - damage[i][q]) / (bytes[i][q] - bytes[i][q-1]), float64; ties: lower
+ * block index; a step that saves no bytes ranks last).  q_out[i] gets the plan, to be
+ * committed with pw_commit_bits at a safe boundary.  Returns PW_ERR_UNSUPPORTED when even
+ * every block at qmin exceeds the budget (q_out then holds qmin).
+ * ------------------------------------------------------------------------------------- */
+pw_status pw_plan_bitwidths(int nblocks, const double* damage, const uint64_t* bytes,
+                            const uint8_t* qmin, const uint8_t* qmax, uint64_t budget,
+                            uint8_t* q_out);
 
 /* ---------------------------------------------------------------------------------------
  * pw_get_status: synchronises `stream`, then returns and clears the device status word of

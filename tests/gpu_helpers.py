@@ -1,6 +1,7 @@
 """Shared helpers of the GPU parity tests (comparison rules and sizes)."""
 import numpy as np
 
+from any_precision_expert_pw_b200 import binding as B
 from any_precision_expert_pw_b200.inputs import CONFIGS
 
 FFN_RTOL_RMS = 2e-3        # max |y_gpu - y_ref| <= 2e-3 * rms(y_ref)
@@ -28,3 +29,24 @@ def assert_ffn_close(y_gpu, y_ref, what=""):
     assert rms > 0, what
     assert err <= FFN_RTOL_RMS * rms, f"{what}: max err {err:.3e} > {FFN_RTOL_RMS} * rms {rms:.3e}"
     return err / rms
+
+
+def tiled_reference(planes, layout):
+    """The tiled arrangement of [n][rows][words] bit-planes, built with array reshapes: row
+    tiles of 32 (gate_up: 16 gate rows then the 16 matching up rows), stages of 32 words, and
+    inside a stage [plane][word pair][row][2]."""
+    n, R, W = planes.shape
+    if layout == B.PW_LAYOUT_TILED_GATE_UP:
+        half = R // 2
+        order = np.concatenate([np.r_[16 * t:16 * t + 16, half + 16 * t:half + 16 * t + 16]
+                                for t in range(half // 16)])
+    else:
+        order = np.arange(R)
+    tiles = planes[:, order, :].reshape(n, R // 32, 32, W)
+    out = []
+    for t in range(R // 32):
+        for s0 in range(0, W, 32):
+            blk = tiles[:, t, :, s0:s0 + 32]                      # [n][32][ws]
+            ws = blk.shape[2]
+            out.append(blk.reshape(n, 32, ws // 2, 2).transpose(0, 2, 1, 3).reshape(-1))
+    return np.concatenate(out)

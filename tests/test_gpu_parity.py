@@ -10,7 +10,7 @@ from any_precision_expert_pw_b200 import binding as B
 from any_precision_expert_pw_b200.inputs import (CONFIGS, MOD_DOWN, MOD_GATE_UP, POLICY_REMAP,
                                                  make_layer, random_indices,
                                                  random_router_inputs)
-from gpu_helpers import GATE_ATOL, SCALED, assert_ffn_close
+from gpu_helpers import GATE_ATOL, SCALED, assert_ffn_close, tiled_reference
 from oracle import bitplanes as obp
 from oracle import ffn as offn
 from oracle import layer as olayer
@@ -31,27 +31,6 @@ def _stream(torch):
 
 
 # ------------------------------------------------------------------ K0 pack
-def tiled_reference(planes, layout):
-    """The tiled arrangement of [n][rows][words] bit-planes, built with array reshapes: row
-    tiles of 32 (gate_up: 16 gate rows then the 16 matching up rows), stages of 32 words, and
-    inside a stage [plane][word pair][row][2]."""
-    n, R, W = planes.shape
-    if layout == B.PW_LAYOUT_TILED_GATE_UP:
-        half = R // 2
-        order = np.concatenate([np.r_[16 * t:16 * t + 16, half + 16 * t:half + 16 * t + 16]
-                                for t in range(half // 16)])
-    else:
-        order = np.arange(R)
-    tiles = planes[:, order, :].reshape(n, R // 32, 32, W)
-    out = []
-    for t in range(R // 32):
-        for s0 in range(0, W, 32):
-            blk = tiles[:, t, :, s0:s0 + 32]                      # [n][32][ws]
-            ws = blk.shape[2]
-            out.append(blk.reshape(n, 32, ws // 2, 2).transpose(0, 2, 1, 3).reshape(-1))
-    return np.concatenate(out)
-
-
 @pytest.mark.parametrize("rows,cols,n", [(32, 128, 4), (96, 4096, 8), (64, 1408, 8), (7, 96, 3)])
 def test_pack_bit_exact(torch_dev, rows, cols, n):
     torch, dev = torch_dev
