@@ -88,20 +88,13 @@ struct Layout {
 
 enum { MODE_GATE_UP = 0, MODE_DOWN = 1 };
 
-struct Params {
-  const pw_page_table* pt;
-  int layer;
-  int E;
-  int mode;      // MODE_GATE_UP or MODE_DOWN
+// One module's half of the launch.
+struct ModeParams {
   int rows;      // expected block rows (2I or H)
   int cols;      // expected block cols (H or I)
   int half;      // gate_up: I (offset of the up rows); down: 0
   int tiles;     // row tiles per expert
   int kslices;   // k-slices per tile (1 for gate_up)
-  const int32_t* counts;
-  const int32_t* offsets;
-  const int32_t* active;
-  const int32_t* meta;
   const float* act;  // [row][ld_act] fp32 activations in xslot order, zero beyond cols
   int ld_act;
   const int32_t* act_map;  // non-null: grouped position pos reads row act_map[pos] / act_div
@@ -109,7 +102,24 @@ struct Params {
   float* out;        // gate_up: h [pos][ld_out] (xslot order); down: [kslice][pos][ld_out]
   int ld_out;
   long long out_slice;  // elements between k-slices of `out`
-  int* sched;           // work counter (zero at launch): items after each CTA's first one
+};
+
+// The launch covers modes first_mode..last_mode: first every gate_up item (expert-major), then
+// every down item.  With both, a down item of active expert a streams h only once done[a]
+// counts all gate_up tiles of a (items are claimed in order and only by running CTAs, none of
+// which waits on a later item, so the wait always ends).
+struct Params {
+  const pw_page_table* pt;
+  int layer;
+  int E;
+  int first_mode, last_mode;
+  ModeParams m[2];
+  const int32_t* counts;
+  const int32_t* offsets;
+  const int32_t* active;
+  const int32_t* meta;
+  int* sched;   // work counter (zero at launch): items after each CTA's first one
+  int* done;    // [E] gate_up tiles finished per active expert (zero at launch), both modes
 };
 
 // One work item as every warp role sees it: written once by LUT warp 0 into a shared-memory
@@ -117,7 +127,7 @@ struct Params {
 struct Desc {
   const uint32_t* planes;  // the tile's run of stages (tiled layout)
   const uint16_t* lut;     // the block's q-bit LUT
-  int item, valid, status, q, n, te, pos0, tile, ks, s0, s1, segA, segB, pad0, pad1, pad2;
+  int item, valid, status, q, n, te, pos0, tile, ks, s0, s1, segA, segB, mode, a, pad0;
 };
 static_assert(sizeof(Desc) == 80, "descriptor size");
 
@@ -125,42 +135,57 @@ struct Item {
   const pw_block* blk;
   const uint16_t* lut;
   const uint32_t* planes;  // the tile's run of stages (tiled layout)
-  int q, n, tile, ks, te, pos0, segA, segB, s0, s1, status;
+  int q, n, tile, ks, te, pos0, segA, segB, s0, s1, status, mode, a;
   bool valid;
 };
 
-__device__ __forceinline__ Item resolve(const Params& p, int item) {
+__device__ __forceinline__ int items_of(const Params& p, int mode, int n_active) {
+  return n_active * p.m[mode].tiles * p.m[mode].kslices;
+}
+
+__device__ __forceinline__ Item resolve(const Params& p, int item, int n_active) {
   Item it;
-  const int per_expert = p.tiles * p.kslices;
+  int mode = p.first_mode;
+  if (mode < p.last_mode) {
+    const int n0 = items_of(p, mode, n_active);
+    if (item >= n0) {
+      item -= n0;
+      ++mode;
+    }
+  }
+  const ModeParams& mp = p.m[mode];
+  it.mode = mode;
+  const int per_expert = mp.tiles * mp.kslices;
   const int a = item / per_expert;
   const int rem = item - a * per_expert;
-  it.tile = rem / p.kslices;
-  it.ks = rem - it.tile * p.kslices;
+  it.a = a;
+  it.tile = rem / mp.kslices;
+  it.ks = rem - it.tile * mp.kslices;
   const int e = p.active[a];
-  it.blk = p.pt->blocks + (static_cast<size_t>(p.layer) * p.E + e) * 2 + p.mode;
+  it.blk = p.pt->blocks + (static_cast<size_t>(p.layer) * p.E + e) * 2 + mode;
   const pw_block* b = it.blk;
   it.q = b->committed_bits;
   it.te = p.counts[e];
   it.pos0 = p.offsets[e];
-  if (p.mode == MODE_GATE_UP) {
+  if (mode == MODE_GATE_UP) {
     it.segA = it.tile * kSegRows;
-    it.segB = p.half + it.tile * kSegRows;
+    it.segB = mp.half + it.tile * kSegRows;
   } else {
     it.segA = it.tile * kRows;
     it.segB = it.segA + kSegRows;
   }
-  const int nst = (p.cols + kStageCols - 1) / kStageCols;
-  it.s0 = (nst * it.ks) / p.kslices;
-  it.s1 = (nst * (it.ks + 1)) / p.kslices;
+  const int nst = (mp.cols + kStageCols - 1) / kStageCols;
+  it.s0 = (nst * it.ks) / mp.kslices;
+  it.s1 = (nst * (it.ks + 1)) / mp.kslices;
   // planes held per (tile, stage) run on the device: all parent_bits, or a paged-in prefix
   it.n = b->stored_bits ? b->stored_bits : b->parent_bits;
   const bool bits_ok = it.q >= b->min_bits && it.q <= it.n && it.n <= b->parent_bits &&
                        it.q >= PW_MIN_BITS &&
                        it.q <= PW_MAX_BITS && b->lut[it.q] != nullptr && b->planes != nullptr;
-  it.planes = b->planes + static_cast<size_t>(it.tile) * it.n * kRows * (p.cols / 32);
-  const int want_layout = p.mode == MODE_GATE_UP ? PW_LAYOUT_TILED_GATE_UP : PW_LAYOUT_TILED_DOWN;
-  const bool shape_ok = static_cast<int>(b->rows) == p.rows &&
-                        static_cast<int>(b->cols) == p.cols && b->layout == want_layout;
+  it.planes = b->planes + static_cast<size_t>(it.tile) * it.n * kRows * (mp.cols / 32);
+  const int want_layout = mode == MODE_GATE_UP ? PW_LAYOUT_TILED_GATE_UP : PW_LAYOUT_TILED_DOWN;
+  const bool shape_ok = static_cast<int>(b->rows) == mp.rows &&
+                        static_cast<int>(b->cols) == mp.cols && b->layout == want_layout;
   const bool resident = b->state == PW_PAGE_GPU;
   it.lut = bits_ok ? b->lut[it.q] : nullptr;
   it.valid = bits_ok && shape_ok && resident;
@@ -174,6 +199,33 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
     *abort_flag = 1;
     return false;
   }
+  return true;
+}
+
+// Bounded wait until *ctr >= target (acquire at GPU scope), then order the async-proxy reads
+// that follow after it; false (PW_ERR_TIMEOUT recorded, abort flag set) when the limit ran out.
+__device__ __forceinline__ int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ bool wait_count(const int* ctr, int target,
+                                           volatile int* abort_flag) {
+  if (ld_acquire(ctr) < target) {
+    const unsigned long long t0 = global_ns();
+    for (uint32_t it = 1;; ++it) {
+      __nanosleep(128);
+      if (ld_acquire(ctr) >= target) break;
+      if (*abort_flag) return false;
+      if ((it & 15u) == 0 && global_ns() - t0 > kWaitLimitNs) {
+        set_status(PW_ERR_TIMEOUT);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+  asm volatile("fence.proxy.async.global;" ::: "memory");
   return true;
 }
 
@@ -457,13 +509,16 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
     mbar_fence_init();
   }
   __syncthreads();
-  // gate_up reads the grouping written by the launch before it; down reads only the page table,
-  // the grouping (complete before gate_up started) and weights until its producer needs h.
-  if (p.mode == MODE_GATE_UP) griddep_wait();
+  // a launch that starts with gate_up reads the grouping written by the launch before it; a
+  // down-only launch reads the page table, the grouping (complete before the gate_up launch
+  // started) and weights until its producer needs h
+  if (p.first_mode == MODE_GATE_UP) griddep_wait();
   griddep_launch();
 
-  const int n_items = p.meta[0] * p.tiles * p.kslices;
-  const int words_total = p.cols / 32;
+  const int n_active = p.meta[0];
+  int n_items = 0;
+  for (int m = p.first_mode; m <= p.last_mode; ++m) n_items += items_of(p, m, n_active);
+  const bool fused = p.first_mode == MODE_GATE_UP && p.last_mode == MODE_DOWN;
 
   uint64_t* const desc_full = red_free + 2;  // [kDescRing] descriptor written (LUT warp 0)
   uint64_t* const desc_free = desc_full + kDescRing;  // [kDescRing] read by producer + reducer
@@ -471,13 +526,14 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
   if (warp == kProducerWarp) {
     // ---------------- producer: one thread streams every stage ----------------
     if (lane != 0) return;
-    if (p.mode == MODE_DOWN) {
+    if (p.first_mode == MODE_DOWN) {
       // while the gate_up grid finishes: this CTA's first item's planes into L2, then wait for h
       if (static_cast<int>(blockIdx.x) < n_items) {
-        const Item cur = resolve(p, blockIdx.x);
+        const Item cur = resolve(p, blockIdx.x, n_active);
+        const int wt = p.m[MODE_DOWN].cols / 32;
         if (cur.valid)
           for (int s = cur.s0; s < cur.s1; ++s) {
-            const int ws = min(kStageWords, words_total - s * kStageWords);
+            const int ws = min(kStageWords, wt - s * kStageWords);
             prefetch_l2(cur.planes + static_cast<size_t>(s) * cur.n * kRows * kStageWords,
                         cur.q * ws * kRows * 4);
           }
@@ -491,13 +547,19 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
       mbar_arrive(&desc_free[j % kDescRing]);
       if (cur.item < 0 || *abort_flag) break;
       if (!cur.valid) continue;
+      const ModeParams& mp = p.m[cur.mode];
+      const int words_total = mp.cols / 32;
+      // fused launch: h of this expert is complete once all its gate_up tiles are counted
+      if (fused && cur.mode == MODE_DOWN &&
+          !wait_count(p.done + cur.a, p.m[MODE_GATE_UP].tiles, abort_flag))
+        break;
       for (int ch = 0; ch < cur.te; ch += NTP) {
         const int ntok = min(NTP, cur.te - ch);
         const float* arow[NTP];
         for (int t = 0; t < ntok; ++t) {
           const int pos = cur.pos0 + ch + t;
-          const int r = p.act_map ? p.act_map[pos] / p.act_div : pos;
-          arow[t] = p.act + static_cast<size_t>(r) * p.ld_act;
+          const int r = mp.act_map ? mp.act_map[pos] / mp.act_div : pos;
+          arow[t] = mp.act + static_cast<size_t>(r) * mp.ld_act;
         }
         for (int s = cur.s0; s < cur.s1; ++s, ++g) {
           const int slot = g % LY::kStages;
@@ -529,8 +591,20 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
       __syncwarp();
       if (lane == 0) mbar_arrive(&desc_free[j % kDescRing]);
       if (it.item < 0 || *abort_flag) break;
-      if (!it.valid) continue;
-      for (int ch = 0; ch < it.te; ch += NTP, ++rc) {
+      const ModeParams& mp = p.m[it.mode];
+      if (!it.valid) {
+        // a block that cannot be read (state, bitwidth or shape): its outputs are zeros
+        if (lane == 0) set_status(it.status);
+        for (int t = 0; t < it.te; ++t) {
+          const size_t row = static_cast<size_t>(it.pos0 + t) * mp.ld_out;
+          if (it.mode == MODE_GATE_UP) {
+            if (lane < kSegRows) mp.out[row + xslot(it.tile * kSegRows + lane)] = 0.f;
+          } else {
+            mp.out[it.ks * mp.out_slice + row + it.tile * kRows + lane] = 0.f;
+          }
+        }
+      }
+      for (int ch = 0; it.valid && ch < it.te; ch += NTP, ++rc) {
         const int ntok = min(NTP, it.te - ch);
         const int par = rc & 1;
         wait_bar(&red_full[par], (rc >> 1) & 1, abort_flag);
@@ -539,19 +613,25 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
           float tot = 0.f;
 #pragma unroll
           for (int w = 0; w < kDecodeWarps; ++w) tot += rb[(w * NTP + t) * 32 + lane];
-          const size_t row = static_cast<size_t>(it.pos0 + ch + t) * p.ld_out;
-          if (p.mode == MODE_GATE_UP) {
+          const size_t row = static_cast<size_t>(it.pos0 + ch + t) * mp.ld_out;
+          if (it.mode == MODE_GATE_UP) {
             const float up = __shfl_down_sync(0xffffffffu, tot, 16);
             if (lane < kSegRows) {
               const float h = tot / (1.0f + expf(-tot)) * up;
-              p.out[row + xslot(it.tile * kSegRows + lane)] = h;
+              mp.out[row + xslot(it.tile * kSegRows + lane)] = h;
             }
           } else {
-            p.out[it.ks * p.out_slice + row + it.tile * kRows + lane] = tot;
+            mp.out[it.ks * mp.out_slice + row + it.tile * kRows + lane] = tot;
           }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&red_free[par]);
+      }
+      if (fused && it.mode == MODE_GATE_UP) {
+        // this tile's h rows are written: make them visible, then count the tile
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) atomicAdd(p.done + it.a, 1);
       }
     }
     return;
@@ -572,7 +652,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
           // the producer and the reducer have read descriptor j - kDescRing from this slot
           wait_bar(&desc_free[j % kDescRing], ((j / kDescRing) & 1) ^ 1, abort_flag);
           if (item < n_items) {
-            const Item it = resolve(p, item);
+            const Item it = resolve(p, item, n_active);
             d.planes = it.planes;
             d.lut = it.lut;
             d.item = item;
@@ -588,6 +668,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
             d.s1 = it.s1;
             d.segA = it.segA;
             d.segB = it.segB;
+            d.mode = it.mode;
+            d.a = it.a;
           } else {
             d.item = -1;
           }
@@ -623,30 +705,18 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
   }
 
   // ---------------- decode warps ----------------
-  const int tid = threadIdx.x;
-  const int ndec = kDecodeWarps * 32;
   uint32_t g = 0, rc = 0;
   for (uint32_t j = 0;; ++j) {
     const uint32_t u = j & 1;
     wait_bar(&lut_ready[u], (j >> 1) & 1, abort_flag);
     const Desc d = cdesc[j % kDescRing];
     if (d.item < 0 || *abort_flag) break;
-    if (!d.valid) {
-      if (tid == 0) set_status(d.status);
-      for (int i = tid; i < d.te * kRows; i += ndec) {
-        const int t = i / kRows, r = i - t * kRows;
-        if (p.mode == MODE_GATE_UP) {
-          if (r < kSegRows)
-            p.out[static_cast<size_t>(d.pos0 + t) * p.ld_out + xslot(d.tile * kSegRows + r)] = 0.f;
-        } else {
-          p.out[d.ks * p.out_slice + static_cast<size_t>(d.pos0 + t) * p.ld_out +
-                d.tile * kRows + r] = 0.f;
-        }
-      }
+    if (!d.valid) {  // the reducer writes this item's zeros
       __syncwarp();
       if (lane == 0) mbar_arrive(&lut_free[u]);
       continue;
     }
+    const int words_total = p.m[d.mode].cols / 32;
     const uint32_t lane_base = u * 128 + lane * 4;
     uint4 reg_lut = make_uint4(0u, 0u, 0u, 0u);
     if (d.q == 3)

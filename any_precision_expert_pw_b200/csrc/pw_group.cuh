@@ -15,7 +15,7 @@ constexpr int kMaxAssign = 8192;  // T * k handled by the single-CTA grouping st
 // assignment), inv[T*k] (assignment -> grouped position, -1 for an invalid expert id),
 // active[E] (experts with work, ascending), meta[0] = number of active experts (0 when the page
 // table does not match (layer, E)), meta[1] = number of valid assignments, meta[2] = 1 for a
-// mismatched table, meta[4] / meta[5] = 0 (the FFN launches' work counters).
+// mismatched table, meta[4] = 0 (the FFN launch's work counter).
 __device__ __forceinline__ void group_block(const pw_page_table* __restrict__ pt, int layer,
                                             const int32_t* __restrict__ idx, int TK, int E,
                                             int32_t* __restrict__ counts,
@@ -58,8 +58,7 @@ __device__ __forceinline__ void group_block(const pw_page_table* __restrict__ pt
     meta[0] = bad ? 0 : na;
     meta[1] = o;
     meta[2] = bad ? 1 : 0;
-    meta[4] = 0;  // work counters of the gate_up and down launches
-    meta[5] = 0;
+    meta[4] = 0;  // work counter of the FFN launch
   }
   __syncthreads();
   for (int e = tid; e < E; e += blockDim.x) {
@@ -94,10 +93,11 @@ __global__ void __launch_bounds__(kGroupThreads) setup_kernel(
     int k, int E, const uint16_t* __restrict__ x, int H, int ldx, int vec, float* __restrict__ X,
     int I, int ldh, float* __restrict__ Hbuf, int32_t* __restrict__ counts,
     int32_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ inv,
-    int32_t* __restrict__ active, int32_t* __restrict__ meta) {
+    int32_t* __restrict__ active, int32_t* __restrict__ meta, int32_t* __restrict__ done) {
   griddep_wait();  // launched as a dependent of whatever precedes it in the stream
   griddep_launch();
   if (blockIdx.x == 0) {
+    for (int e = threadIdx.x; e < E; e += blockDim.x) done[e] = 0;
     group_block(pt, layer, idx, T * k, E, counts, offsets, perm, inv, active, meta);
     return;
   }

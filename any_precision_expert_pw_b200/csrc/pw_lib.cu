@@ -75,7 +75,7 @@ pw_status device_info(DeviceInfo** out) {
 
 // Workspace layout of pw_moe_anyprec_forward.
 struct Workspace {
-  size_t counts, offsets, perm, inv, active, meta, X, Hbuf, O, total;
+  size_t counts, offsets, perm, inv, active, meta, done, X, Hbuf, O, total;
   int ldx, ldh;
 };
 
@@ -95,7 +95,8 @@ Workspace ws_layout(int T, int k, int E, int H, int I) {
   w.perm = take(4 * TK);
   w.inv = take(4 * TK);
   w.active = take(4 * static_cast<size_t>(E));
-  w.meta = take(32);  // [0] active experts, [1] valid assignments, [2] bad table, [4..5] work counters
+  w.meta = take(32);  // [0] active experts, [1] valid assignments, [2] bad table, [4] work counter
+  w.done = take(4 * static_cast<size_t>(E));  // gate_up tiles finished per active expert
   w.X = take(4 * static_cast<size_t>(T) * w.ldx);
   w.Hbuf = take(4 * TK * w.ldh);
   w.O = take(4 * TK * H * static_cast<size_t>(pw::k4::kMaxKSlices));
@@ -149,7 +150,9 @@ pw_status launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size
 
 pw_status launch_ffn(const pw::k4::Params& p, int max_active, int ntp, int sms,
                      cudaStream_t st) {
-  const long long items = static_cast<long long>(max_active) * p.tiles * p.kslices;
+  long long items = 0;
+  for (int m = p.first_mode; m <= p.last_mode; ++m)
+    items += static_cast<long long>(max_active) * p.m[m].tiles * p.m[m].kslices;
   const int grid = static_cast<int>(items < sms ? items : sms);
   if (ntp == 1)
     return launch_dependent(pw::k4::ffn_kernel<1>, dim3(grid), dim3(pw::k4::kThreads),
@@ -229,6 +232,7 @@ pw_status pw_moe_anyprec_forward(const pw_page_table* pt_dev, int layer, int E,
   int32_t* inv = reinterpret_cast<int32_t*>(base + w.inv);
   int32_t* active = reinterpret_cast<int32_t*>(base + w.active);
   int32_t* meta = reinterpret_cast<int32_t*>(base + w.meta);
+  int32_t* done = reinterpret_cast<int32_t*>(base + w.done);
   float* X = reinterpret_cast<float*>(base + w.X);
   float* Hb = reinterpret_cast<float*>(base + w.Hbuf);
   float* O = reinterpret_cast<float*>(base + w.O);
@@ -243,7 +247,7 @@ pw_status pw_moe_anyprec_forward(const pw_page_table* pt_dev, int layer, int E,
     const int vec = (reinterpret_cast<uintptr_t>(x_bf16) % 16) == 0;
     if (launch_dependent(pw::setup_kernel, dim3(grid), dim3(pw::kGroupThreads), 0, st, pt_dev,
                          layer, idx, T, k, E, x_bf16, H, w.ldx, vec, X, I, w.ldh, Hb, counts,
-                         offsets, perm, inv, active, meta) != PW_OK)
+                         offsets, perm, inv, active, meta, done) != PW_OK)
       return PW_ERR_CUDA;
   }
   const int max_active = E < TK ? E : TK;
@@ -255,45 +259,47 @@ pw_status pw_moe_anyprec_forward(const pw_page_table* pt_dev, int layer, int E,
   p.offsets = offsets;
   p.active = active;
   p.meta = meta;
-  // gate_up: h = SiLU(W_gate x) * (W_up x)
-  p.mode = pw::k4::MODE_GATE_UP;
-  p.rows = 2 * I;
-  p.cols = H;
-  p.half = I;
-  p.tiles = I / pw::k4::kSegRows;
-  p.kslices = 1;
   p.sched = meta + 4;
-  p.act = X;
-  p.ld_act = w.ldx;
-  p.act_map = perm;  // grouped position -> assignment t*k+slot -> token row of X
-  p.act_div = k;
-  p.out = Hb;
-  p.ld_out = w.ldh;
-  p.out_slice = 0;
+  p.done = done;
+  // one launch: every gate_up item (h = SiLU(W_gate x) * (W_up x)), then every down item
+  // (o = W_down h, split along k so that the work items fill the GPU); a down item streams h
+  // once all gate_up tiles of its expert are counted
+  p.first_mode = pw::k4::MODE_GATE_UP;
+  p.last_mode = pw::k4::MODE_DOWN;
+  pw::k4::ModeParams& gu = p.m[pw::k4::MODE_GATE_UP];
+  gu.rows = 2 * I;
+  gu.cols = H;
+  gu.half = I;
+  gu.tiles = I / pw::k4::kSegRows;
+  gu.kslices = 1;
+  gu.act = X;
+  gu.ld_act = w.ldx;
+  gu.act_map = perm;  // grouped position -> assignment t*k+slot -> token row of X
+  gu.act_div = k;
+  gu.out = Hb;
+  gu.ld_out = w.ldh;
+  gu.out_slice = 0;
+  pw::k4::ModeParams& dn = p.m[pw::k4::MODE_DOWN];
+  dn.rows = H;
+  dn.cols = I;
+  dn.half = 0;
+  dn.tiles = H / pw::k4::kRows;
+  dn.kslices = choose_kslices(max_active * dn.tiles,
+                              (I + pw::k4::kStageCols - 1) / pw::k4::kStageCols, di->sms);
+  dn.act = Hb;
+  dn.ld_act = w.ldh;
+  dn.act_map = nullptr;
+  dn.act_div = 1;
+  dn.out = O;
+  dn.ld_out = H;
+  dn.out_slice = static_cast<long long>(TK) * H;
   const int ntp = T == 1 ? 1 : (T == 2 ? 2 : 4);
-  if (launch_ffn(p, max_active, ntp, di->sms, st) != PW_OK) return PW_ERR_CUDA;
-  // down: o = W_down h, split along k so that the grid fills the GPU
-  p.mode = pw::k4::MODE_DOWN;
-  p.rows = H;
-  p.cols = I;
-  p.half = 0;
-  p.tiles = H / pw::k4::kRows;
-  p.kslices = choose_kslices(max_active * p.tiles, (I + pw::k4::kStageCols - 1) / pw::k4::kStageCols,
-                             di->sms);
-  p.sched = meta + 5;
-  p.act = Hb;
-  p.ld_act = w.ldh;
-  p.act_map = nullptr;
-  p.act_div = 1;
-  p.out = O;
-  p.ld_out = H;
-  p.out_slice = static_cast<long long>(TK) * H;
   if (launch_ffn(p, max_active, ntp, di->sms, st) != PW_OK) return PW_ERR_CUDA;
   {
     const dim3 g((H + 255) / 256, T);
     return launch_dependent(pw::combine_kernel, g, dim3(256), 0, st,
                             static_cast<const float*>(O), static_cast<const int32_t*>(inv), gate,
-                            static_cast<const int32_t*>(meta), T, k, H, p.kslices,
+                            static_cast<const int32_t*>(meta), T, k, H, dn.kslices,
                             static_cast<long long>(TK) * H, y);
   }
 }

@@ -329,8 +329,8 @@ def run_pw(args):
     with torch.cuda.graph(g_ffn, stream=stream):
         D.ffn()
     # router (+ top-k, fused into it when the E experts fit one CTA of 8), the assignment
-    # rewrite if any, then setup, gate_up, down and combine
-    launches_step = (1 if cfg.E <= 8 else 2) + (0 if cfg.policy == POLICY_NONE else 1) + 4
+    # rewrite if any, then setup, the FFN (gate_up and down in one launch) and combine
+    launches_step = (1 if cfg.E <= 8 else 2) + (0 if cfg.policy == POLICY_NONE else 1) + 3
 
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(int(2.5 * l2), dtype=torch.uint8, device=dev)
