@@ -40,7 +40,8 @@ EXPORTS = ("pw_block_prepare", "pw_pack_bitplanes", "pw_route_topk", "pw_topk", 
            "pw_plan_bitwidths",
            "pw_moe_workspace_bytes",
            "pw_moe_anyprec_forward",
-           "pw_moe_anyprec_forward_static", "pw_commit_bits", "pw_get_status",
+           "pw_moe_anyprec_forward_static", "pw_set_tc_min_tokens", "pw_commit_bits",
+           "pw_get_status",
            "pw_status_string", "pw_version")
 PW_STATIC_WORKSPACE_BYTES = 16 << 20
 
@@ -107,6 +108,7 @@ def lib() -> ctypes.CDLL:
         L.pw_moe_workspace_bytes.restype = Z
         L.pw_moe_anyprec_forward.argtypes = [P, I, I, P, I, I, I, I, P, P, P, P, Z, S]
         L.pw_moe_anyprec_forward_static.argtypes = [P, I, I, P, I, I, I, I, P, P, P, S]
+        L.pw_set_tc_min_tokens.argtypes = [I]
         L.pw_commit_bits.argtypes = [P, I, P, P, I, S]
         L.pw_page_copy.argtypes = [P, I, P, I, I, I, I, S]
         L.pw_page_update.argtypes = [P, I, P, I, S]
@@ -202,6 +204,10 @@ def pw_moe_anyprec_forward_static(pt_dev, layer, E, x_bf16, T, H, I, k, idx, gat
     workspace, for callers that cannot allocate device memory (see include/pw.h)."""
     return lib().pw_moe_anyprec_forward_static(pt_dev, layer, E, x_bf16, T, H, I, k, idx, gate,
                                                y, stream)
+
+
+def pw_set_tc_min_tokens(tokens_per_expert) -> int:
+    return lib().pw_set_tc_min_tokens(tokens_per_expert)
 
 
 def pw_commit_bits(pt_dev, num_blocks, block_ids, q, count, stream=0) -> int:

@@ -10,14 +10,35 @@ namespace pw {
 
 constexpr int kGroupThreads = 1024;
 constexpr int kMaxAssign = 8192;  // T * k handled by the single-CTA grouping step
+constexpr int kPassTokens = 64;   // tokens of one expert per tensor-core pass (MMA N <= 64)
+
+// What the tensor-core FFN needs beyond the plain grouping.  Each expert's tokens are split
+// into passes of up to kPassTokens; a pass of m tokens is padded to np = m rounded up to 16
+// (the MMA's N).  Padded rows: expert e owns rows [pbase[e], pbase[e] + roundup16(count)),
+// pass j of it rows pbase[e] + 64j ..; ptok[row] = token of the row (-1 for padding),
+// pnn[row] = np << 16 | (row - first row of its pass); pass_tab[i] = a | j << 16 for the i-th
+// (active expert a, pass j) in ascending (a, j); meta[5] = number of passes, meta[6] = number
+// of padded rows.
+struct PassOut {
+  int32_t* pbase;     // [E]
+  int32_t* ptok;      // [padded rows]
+  int32_t* pnn;       // [padded rows]
+  int32_t* pass_tab;  // [E + T*k/64 + 1]
+};
+
+__host__ __device__ __forceinline__ int pass_np(int count, int j) {
+  const int m = min(kPassTokens, count - kPassTokens * j);
+  return (m + 15) & ~15;
+}
 
 // Grouping, run by one CTA.  counts[E], offsets[E+1], perm[T*k] (grouped position ->
 // assignment), inv[T*k] (assignment -> grouped position, -1 for an invalid expert id),
 // active[E] (experts with work, ascending), meta[0] = number of active experts (0 when the page
 // table does not match (layer, E)), meta[1] = number of valid assignments, meta[2] = 1 for a
-// mismatched table, meta[4] = 0 (the FFN launch's work counter).
+// mismatched table, meta[4] = 0 (the FFN launch's work counter); and the PassOut arrays.
 __device__ __forceinline__ void group_block(const pw_page_table* __restrict__ pt, int layer,
-                                            const int32_t* __restrict__ idx, int TK, int E,
+                                            const int32_t* __restrict__ idx, int TK, int k,
+                                            int E, const PassOut& po,
                                             int32_t* __restrict__ counts,
                                             int32_t* __restrict__ offsets,
                                             int32_t* __restrict__ perm, int32_t* __restrict__ inv,
@@ -26,6 +47,7 @@ __device__ __forceinline__ void group_block(const pw_page_table* __restrict__ pt
   __shared__ int cnt[PW_MAX_EXPERTS];
   __shared__ int off[PW_MAX_EXPERTS + 1];
   __shared__ int act_pos[PW_MAX_EXPERTS + 1];
+  __shared__ int pb[PW_MAX_EXPERTS];
   __shared__ int16_t eid[kMaxAssign];
   const int tid = threadIdx.x;
   for (int e = tid; e < E; e += blockDim.x) cnt[e] = 0;
@@ -46,11 +68,15 @@ __device__ __forceinline__ void group_block(const pw_page_table* __restrict__ pt
                      static_cast<int>(pt->num_experts) != E ||
                      (reinterpret_cast<uintptr_t>(pt->blocks) & 63) != 0;
     if (bad) set_status(PW_ERR_INVALID_ARG);
-    int o = 0, na = 0;
+    int o = 0, na = 0, prow = 0, npass = 0;
     for (int e = 0; e < E; ++e) {
       off[e] = o;
       act_pos[e] = na;
+      pb[e] = prow;
+      if (cnt[e] > 0 && !bad)
+        for (int j = 0; j * kPassTokens < cnt[e]; ++j) po.pass_tab[npass++] = na | (j << 16);
       o += cnt[e];
+      prow += (cnt[e] + 15) & ~15;
       na += (cnt[e] > 0);
     }
     off[E] = o;
@@ -59,12 +85,19 @@ __device__ __forceinline__ void group_block(const pw_page_table* __restrict__ pt
     meta[1] = o;
     meta[2] = bad ? 1 : 0;
     meta[4] = 0;  // work counter of the FFN launch
+    meta[5] = npass;
+    meta[6] = prow;
   }
   __syncthreads();
   for (int e = tid; e < E; e += blockDim.x) {
     counts[e] = cnt[e];
     offsets[e] = off[e];
+    po.pbase[e] = pb[e];
     if (cnt[e] > 0) active[act_pos[e]] = e;
+    for (int r = cnt[e]; r < ((cnt[e] + 15) & ~15); ++r) {  // padding rows of the last pass
+      po.ptok[pb[e] + r] = -1;
+      po.pnn[pb[e] + r] = (pass_np(cnt[e], r / kPassTokens) << 16) | (r % kPassTokens);
+    }
   }
   if (tid == 0) offsets[E] = off[E];
   for (int a = tid; a < TK; a += blockDim.x) {
@@ -78,6 +111,8 @@ __device__ __forceinline__ void group_block(const pw_page_table* __restrict__ pt
     const int pos = off[e] + r;
     perm[pos] = a;
     inv[a] = pos;
+    po.ptok[pb[e] + r] = a / k;
+    po.pnn[pb[e] + r] = (pass_np(cnt[e], r / kPassTokens) << 16) | (r % kPassTokens);
   }
 }
 
@@ -88,17 +123,20 @@ __device__ __forceinline__ void group_block(const pw_page_table* __restrict__ pt
 // padding must read as zero, and it reads activations in its decode order (xslot, a
 // permutation inside each 32-column group that keeps padding groups whole).  `vec`: x is
 // 16-byte aligned (H is a multiple of 128), so a thread converts 8 columns from one load.
+// The tensor-core FFN stages its activations with stage_x_kernel instead; it launches this
+// kernel with CTA 0 alone.
 __global__ void __launch_bounds__(kGroupThreads) setup_kernel(
     const pw_page_table* __restrict__ pt, int layer, const int32_t* __restrict__ idx, int T,
     int k, int E, const uint16_t* __restrict__ x, int H, int ldx, int vec, float* __restrict__ X,
     int I, int ldh, float* __restrict__ Hbuf, int32_t* __restrict__ counts,
     int32_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ inv,
-    int32_t* __restrict__ active, int32_t* __restrict__ meta, int32_t* __restrict__ done) {
+    int32_t* __restrict__ active, int32_t* __restrict__ meta, int32_t* __restrict__ done,
+    PassOut po) {
   griddep_wait();  // launched as a dependent of whatever precedes it in the stream
   griddep_launch();
   if (blockIdx.x == 0) {
     for (int e = threadIdx.x; e < E; e += blockDim.x) done[e] = 0;
-    group_block(pt, layer, idx, T * k, E, counts, offsets, perm, inv, active, meta);
+    group_block(pt, layer, idx, T * k, k, E, po, counts, offsets, perm, inv, active, meta);
     return;
   }
   const size_t nthr = static_cast<size_t>(gridDim.x - 1) * blockDim.x;
@@ -136,6 +174,56 @@ __global__ void __launch_bounds__(kGroupThreads) setup_kernel(
       const size_t pos = i / padh;
       Hbuf[pos * ldh + I + (i - pos * padh)] = 0.0f;
     }
+  }
+}
+
+// The tensor-core FFN's gate_up operand: for every padded row (ptok, pnn as in PassOut) the
+// token's activations as fp16, in the MMA's K-major core-matrix order per 128-column chunk:
+// element (n, c) of the pass starting at padded row r0 (np rows) sits at
+//   r0 * H + (c / 128) * np * 128 + ((c % 128) / 8) * np * 8 + n * 8 + c % 8
+// (so one chunk of a pass is np * 256 contiguous bytes); padding rows are zeros.  bf16 -> fp16
+// is exact for values in fp16's normal range.  `vec`: x is 16-byte aligned.
+__global__ void __launch_bounds__(256) stage_x_kernel(const uint16_t* __restrict__ x, int H,
+                                                      int vec, const int32_t* __restrict__ ptok,
+                                                      const int32_t* __restrict__ pnn,
+                                                      const int32_t* __restrict__ meta,
+                                                      __half* __restrict__ XB) {
+  griddep_wait();  // grouping of the launch before
+  griddep_launch();
+  const int rows = meta[6];
+  const int g8 = H / 8;
+  const size_t n_all = static_cast<size_t>(rows) * g8;
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_all;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int row = static_cast<int>(i / g8);
+    const int c = static_cast<int>(i - static_cast<size_t>(row) * g8) * 8;
+    const int tok = ptok[row];
+    const int nn = pnn[row];
+    const int np = nn >> 16, n = nn & 0xffff;
+    __half* dst = XB + static_cast<size_t>(row - n) * H + (c / 128) * np * 128 +
+                  ((c % 128) / 8) * np * 8 + n * 8;
+    uint4 out = make_uint4(0u, 0u, 0u, 0u);
+    if (tok >= 0) {
+      const uint16_t* src = x + static_cast<size_t>(tok) * H + c;
+      uint32_t w[4];
+      if (vec) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(src));
+        w[0] = u.x; w[1] = u.y; w[2] = u.z; w[3] = u.w;
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          w[j] = static_cast<uint32_t>(src[2 * j]) | (static_cast<uint32_t>(src[2 * j + 1]) << 16);
+      }
+      uint32_t o[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const __half2 h = __floats2half2_rn(__uint_as_float(w[j] << 16),
+                                            __uint_as_float(w[j] & 0xffff0000u));
+        o[j] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+      out = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    *reinterpret_cast<uint4*>(dst) = out;
   }
 }
 

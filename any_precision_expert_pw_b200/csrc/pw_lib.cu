@@ -7,6 +7,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <atomic>
 #include <mutex>
 #include <queue>
 #include <vector>
@@ -19,6 +20,7 @@
 #include "pw_pack.cuh"
 #include "pw_route.cuh"
 #include "pw_table.cuh"
+#include "pw_tc.cuh"
 
 static_assert(sizeof(pw_block) == 256, "pw_block layout");
 static_assert(offsetof(pw_block, planes) == 16, "pw_block layout");
@@ -65,7 +67,9 @@ pw_status device_info(DeviceInfo** out) {
         cudaFuncSetAttribute(pw::k4::ffn_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              pw::k4::Layout<2>::kSmem) != cudaSuccess ||
         cudaFuncSetAttribute(pw::k4::ffn_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             pw::k4::Layout<4>::kSmem) != cudaSuccess)
+                             pw::k4::Layout<4>::kSmem) != cudaSuccess ||
+        cudaFuncSetAttribute(pw::k5::tc_ffn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             pw::k5::kSmem) != cudaSuccess)
       return PW_ERR_CUDA;
     d.ffn_attr_set = true;
   }
@@ -75,7 +79,8 @@ pw_status device_info(DeviceInfo** out) {
 
 // Workspace layout of pw_moe_anyprec_forward.
 struct Workspace {
-  size_t counts, offsets, perm, inv, active, meta, done, X, Hbuf, O, total;
+  size_t counts, offsets, perm, inv, active, meta, done, X, Hbuf, O;
+  size_t pbase, ptok, pnn, pass_tab, XB, HB, total;  // tensor-core path
   int ldx, ldh;
 };
 
@@ -100,6 +105,14 @@ Workspace ws_layout(int T, int k, int E, int H, int I) {
   w.X = take(4 * static_cast<size_t>(T) * w.ldx);
   w.Hbuf = take(4 * TK * w.ldh);
   w.O = take(4 * TK * H * static_cast<size_t>(pw::k4::kMaxKSlices));
+  // tensor-core path: each active expert's rows padded to a multiple of 16
+  const size_t rows_pad = TK + 15 * std::min<size_t>(E, TK);
+  w.pbase = take(4 * static_cast<size_t>(E));
+  w.ptok = take(4 * rows_pad);
+  w.pnn = take(4 * rows_pad);
+  w.pass_tab = take(4 * (std::min<size_t>(E, TK) + TK / pw::kPassTokens + 1));
+  w.XB = take(2 * rows_pad * H);
+  w.HB = take(2 * rows_pad * I);
   w.total = o;
   return w;
 }
@@ -111,6 +124,9 @@ static __device__ __align__(256) uint8_t g_static_ws[PW_STATIC_WORKSPACE_BYTES];
 void* g_static_ws_addr[kMaxDevices] = {};
 std::mutex g_static_ws_mu;
 
+
+// Average routed tokens per active expert from which the tensor-core FFN is used.
+std::atomic<int> g_tc_min_tokens{8};
 
 // k-slices for the down projection: fill the GPU in whole waves of work items, with at least
 // two 1024-column stages per slice.
@@ -237,20 +253,86 @@ pw_status pw_moe_anyprec_forward(const pw_page_table* pt_dev, int layer, int E,
   float* Hb = reinterpret_cast<float*>(base + w.Hbuf);
   float* O = reinterpret_cast<float*>(base + w.O);
   const int TK = T * k;
+  const int max_active = E < TK ? E : TK;
+  // tensor-core FFN once the batch routes enough tokens to each expert
+  const bool use_tc = static_cast<long long>(TK) >=
+                      static_cast<long long>(g_tc_min_tokens.load()) * max_active;
+  pw::PassOut po;
+  po.pbase = reinterpret_cast<int32_t*>(base + w.pbase);
+  po.ptok = reinterpret_cast<int32_t*>(base + w.ptok);
+  po.pnn = reinterpret_cast<int32_t*>(base + w.pnn);
+  po.pass_tab = reinterpret_cast<int32_t*>(base + w.pass_tab);
+  const int vec = (reinterpret_cast<uintptr_t>(x_bf16) % 16) == 0;
 
   {
-    // CTA 0 groups; the others convert x (8 columns per thread)
+    // CTA 0 groups; the others convert x (8 columns per thread) for the CUDA-core FFN
     const long long groups = static_cast<long long>(T) * (w.ldx / 8) +
                              static_cast<long long>(TK) * (w.ldh - I) / 8;
     const long long conv = (groups + pw::kGroupThreads - 1) / pw::kGroupThreads;
-    const int grid = 1 + static_cast<int>(std::min<long long>(std::max(conv, 1LL), 2LL * di->sms));
-    const int vec = (reinterpret_cast<uintptr_t>(x_bf16) % 16) == 0;
+    const int grid =
+        use_tc ? 1 : 1 + static_cast<int>(std::min<long long>(std::max(conv, 1LL), 2LL * di->sms));
     if (launch_dependent(pw::setup_kernel, dim3(grid), dim3(pw::kGroupThreads), 0, st, pt_dev,
                          layer, idx, T, k, E, x_bf16, H, w.ldx, vec, X, I, w.ldh, Hb, counts,
-                         offsets, perm, inv, active, meta, done) != PW_OK)
+                         offsets, perm, inv, active, meta, done, po) != PW_OK)
       return PW_ERR_CUDA;
   }
-  const int max_active = E < TK ? E : TK;
+  if (use_tc) {
+    __half* XB = reinterpret_cast<__half*>(base + w.XB);
+    __half* HB = reinterpret_cast<__half*>(base + w.HB);
+    {
+      const long long rows_pad = TK + 15LL * max_active;
+      const long long n = rows_pad * (H / 8);
+      const int grid = static_cast<int>(std::min<long long>((n + 255) / 256, 4LL * di->sms));
+      if (launch_dependent(pw::stage_x_kernel, dim3(grid), dim3(256), 0, st, x_bf16, H, vec,
+                           static_cast<const int32_t*>(po.ptok),
+                           static_cast<const int32_t*>(po.pnn),
+                           static_cast<const int32_t*>(meta), XB) != PW_OK)
+        return PW_ERR_CUDA;
+    }
+    pw::k5::Params q;
+    q.pt = pt_dev;
+    q.layer = layer;
+    q.E = E;
+    q.counts = counts;
+    q.offsets = offsets;
+    q.active = active;
+    q.meta = meta;
+    q.pbase = po.pbase;
+    q.pass_tab = po.pass_tab;
+    q.sched = meta + 4;
+    q.done = done;
+    pw::k5::ModeParams& gu = q.m[pw::k5::MODE_GATE_UP];
+    gu.rows = 2 * I;
+    gu.cols = H;
+    gu.half = I;
+    gu.mblocks = I / 64;  // four 16-row gate/up tile pairs per block
+    gu.kslices = 1;
+    gu.bsrc = XB;
+    gu.hout = HB;
+    gu.out = nullptr;
+    gu.ld_out = 0;
+    gu.out_slice = 0;
+    pw::k5::ModeParams& dn = q.m[pw::k5::MODE_DOWN];
+    dn.rows = H;
+    dn.cols = I;
+    dn.half = 0;
+    dn.mblocks = H / pw::k5::kRows;
+    dn.kslices = choose_kslices(max_active * dn.mblocks,
+                                (I + pw::k4::kStageCols - 1) / pw::k4::kStageCols, di->sms);
+    dn.bsrc = HB;
+    dn.hout = nullptr;
+    dn.out = O;
+    dn.ld_out = H;
+    dn.out_slice = static_cast<long long>(TK) * H;
+    if (launch_dependent(pw::k5::tc_ffn_kernel, dim3(di->sms), dim3(pw::k5::kThreads),
+                         pw::k5::kSmem, st, q) != PW_OK)
+      return PW_ERR_CUDA;
+    const dim3 g((H + 255) / 256, T);
+    return launch_dependent(pw::combine_kernel, g, dim3(256), 0, st,
+                            static_cast<const float*>(O), static_cast<const int32_t*>(inv), gate,
+                            static_cast<const int32_t*>(meta), T, k, H, dn.kslices,
+                            static_cast<long long>(TK) * H, y);
+  }
   pw::k4::Params p;
   p.pt = pt_dev;
   p.layer = layer;
@@ -325,6 +407,12 @@ pw_status pw_moe_anyprec_forward_static(const pw_page_table* pt_dev, int layer, 
   }
   return pw_moe_anyprec_forward(pt_dev, layer, E, x_bf16, T, H, I, k, idx, gate, y, ws, need,
                                 stream);
+}
+
+pw_status pw_set_tc_min_tokens(int tokens_per_expert) {
+  if (tokens_per_expert < 0) return PW_ERR_INVALID_ARG;
+  g_tc_min_tokens.store(tokens_per_expert);
+  return PW_OK;
 }
 
 pw_status pw_commit_bits(pw_page_table* pt_dev, int num_blocks, const int32_t* block_ids,

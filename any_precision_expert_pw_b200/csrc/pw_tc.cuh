@@ -1,0 +1,663 @@
+// K5: the grouped expert FFN for larger batches, on the tensor cores (PagedWeight, "Composants
+// Clés" 1 and 3: one fused kernel reads the bit-planes and LUTs directly, each block at its own
+// bitwidth).  With many tokens per expert the bit-plane GEMV of K4, which decodes every weight
+// once per four tokens, becomes a GEMM: here each weight is decoded once per pass of up to 64
+// tokens and the products run on tcgen05.
+//
+// Work item = (active expert, pass of up to 64 of its tokens, 128-row block = four 32-row
+// tiles, k-slice).  D[128 rows][np tokens] (fp32, in tensor memory) += A[128][K] * B[np][K]^T,
+// with A the decoded weights (fp16 LUT values, exact) and B the pass's activations (fp16).
+//
+// Warp roles (one CTA per SM, persistent over the items):
+//   decode (16 warps)      warp w takes tile w % 4 of the block and word w / 4 of each
+//                          128-column chunk; lane = row.  An 8x8 bit transpose of its q plane
+//                          words gives one code byte per weight, a gather from the row's table
+//                          gives the fp16 value, and the 32 values go to the chunk's A buffer
+//                          in the MMA's K-major core-matrix order;
+//   table/epilogue (4)     warp 16 + j: builds the decode table of tile j's 32 rows for every
+//                          item, and reads rows 32j.. of the accumulator back (tensor-memory lane
+//                          quarter j) for the epilogue: SiLU(gate) * up as fp16 into the down
+//                          projection's operand, or the down rows into the k-slice partials;
+//                          warp 16 also takes the items (first blockIdx.x, then a work counter);
+//   plane producer (1)     bulk-copies each chunk's top-q planes of the four tiles (4q runs of
+//                          512 bytes in the tiled layout) into a ring of four stages;
+//   operand producer (1)   bulk-copies each chunk's activations (np * 256 contiguous bytes);
+//                          a down item first waits until every gate_up item of its expert is
+//                          counted;
+//   MMA (1)                one thread issues 8 tcgen05.mma (K = 16 each) per chunk into one of
+//                          two accumulators and commits each chunk's completion to the barrier
+//                          that frees its A and B buffers.
+// The decode table holds, for row r, slot u = (LUT[2u], LUT[2u+1]) at byte 512u + 4r, so a
+// warp's gathers hit 32 different banks; the code's low bit picks the half.
+#pragma once
+#include "pw_common.cuh"
+#include "pw_ffn.cuh"
+#include "pw_group.cuh"
+
+namespace pw {
+namespace k5 {
+
+constexpr int kRows = 128;        // MMA M
+constexpr int kTiles = 4;         // 32-row tiles per item
+constexpr int kChunkCols = 128;   // K columns per pipeline step
+constexpr int kPass = kPassTokens;
+constexpr int kDecodeWarps = 16;
+constexpr int kEpiWarp0 = 16;
+constexpr int kEpiWarps = 4;
+constexpr int kPlaneWarp = 20;
+constexpr int kOperandWarp = 21;
+constexpr int kMmaWarp = 22;
+constexpr int kThreads = 23 * 32;
+constexpr int kTmemCols = 2 * kPass;  // two accumulators of up to 64 fp32 columns
+constexpr int kPlaneStages = 4;
+constexpr int kDescRing = 8;
+
+constexpr int kOffTable = 0;
+constexpr int kTableBytes = 128 * kRows * 4;            // 2^8 / 2 slots x 128 rows x 4 bytes
+constexpr int kOffA = kOffTable + kTableBytes;
+constexpr int kABytes = (kChunkCols / 8) * kRows * 16;  // [16 k-groups][128 rows][16 bytes]
+constexpr int kOffB = kOffA + 2 * kABytes;
+constexpr int kBBytes = (kChunkCols / 8) * kPass * 16;  // [16 k-groups][np rows][16 bytes]
+constexpr int kOffPlanes = kOffB + 2 * kBBytes;
+constexpr int kPieceBytes = 512;                        // one plane of one tile for one chunk
+constexpr int kPlaneStageBytes = kTiles * PW_MAX_BITS * kPieceBytes;
+constexpr int kOffDesc = kOffPlanes + kPlaneStages * kPlaneStageBytes;
+
+enum { MODE_GATE_UP = 0, MODE_DOWN = 1 };
+
+struct ModeParams {
+  int rows;      // expected block rows (2I or H)
+  int cols;      // expected block cols (H or I)
+  int half;      // gate_up: I (offset of the up rows); down: 0
+  int mblocks;   // 128-row blocks per expert
+  int kslices;   // k-slices per block (1 for gate_up)
+  const __half* bsrc;  // operand staging [padded rows][cols], chunk order (stage_x_kernel)
+  __half* hout;        // gate_up: the down projection's operand staging [padded rows][I]
+  float* out;          // down: [kslice][pos][ld_out]
+  int ld_out;
+  long long out_slice;
+};
+
+// gate_up items: passes x gate_up blocks; then down items: passes x down blocks x k-slices.
+struct Params {
+  const pw_page_table* pt;
+  int layer;
+  int E;
+  ModeParams m[2];
+  const int32_t* counts;
+  const int32_t* offsets;
+  const int32_t* active;
+  const int32_t* meta;
+  const int32_t* pbase;
+  const int32_t* pass_tab;
+  int* sched;  // work counter (zero at launch)
+  int* done;   // [E] per active expert: gate_up items finished x 4 epilogue warps (zero at launch)
+};
+
+struct Desc {
+  const uint32_t* planes;  // tile 0 of the block (tiled layout); tiles follow at tile_words
+  const uint16_t* lut;     // the block's q-bit LUT
+  const __half* bsrc;      // chunk 0 of this pass's operand
+  long long tile_words;
+  int item, valid, status, q, n, mode, a, mb, ks, c0, c1, np, te, pos0, prow0, target;
+};
+static_assert(sizeof(Desc) == 96, "descriptor size");
+
+constexpr int kOffBar = kOffDesc + kDescRing * static_cast<int>(sizeof(Desc));
+// barriers: pl_full[4] pl_empty[4] b_full[2] ab_empty[2] a_full[2] acc_full[2] acc_empty[2]
+// table_ready table_free desc_full[8] desc_free[8] mma_done; then the TMEM address and abort
+constexpr int kNumBars = 2 * kPlaneStages + 10 + 2 + 2 * kDescRing + 1;
+constexpr int kSmem = kOffBar + kNumBars * 8 + 16;
+static_assert(kSmem <= 227 * 1024, "shared memory budget");
+static_assert(kOffA % 1024 == 0 && kOffB % 1024 == 0 && kOffPlanes % 1024 == 0, "alignment");
+
+__device__ __forceinline__ int items_of(const Params& p, int mode, int npass) {
+  return npass * p.m[mode].mblocks * p.m[mode].kslices;
+}
+
+__device__ __forceinline__ Desc resolve(const Params& p, int item, int npass) {
+  Desc d;
+  int mode = MODE_GATE_UP;
+  const int n0 = items_of(p, MODE_GATE_UP, npass);
+  if (item >= n0) {
+    item -= n0;
+    mode = MODE_DOWN;
+  }
+  const ModeParams& mp = p.m[mode];
+  const int per_pass = mp.mblocks * mp.kslices;
+  const int pi = item / per_pass;
+  const int rem = item - pi * per_pass;
+  d.mb = rem / mp.kslices;
+  d.ks = rem - d.mb * mp.kslices;
+  const int pt_ent = p.pass_tab[pi];
+  const int a = pt_ent & 0xffff, j = pt_ent >> 16;
+  const int e = p.active[a];
+  const int cnt = p.counts[e];
+  d.mode = mode;
+  d.a = a;
+  d.te = min(kPass, cnt - kPass * j);
+  d.np = pass_np(cnt, j);
+  d.pos0 = p.offsets[e] + kPass * j;
+  d.prow0 = p.pbase[e] + kPass * j;
+  // each of the four epilogue warps counts every gate_up item of the expert once
+  d.target = kEpiWarps * p.m[MODE_GATE_UP].mblocks * ((cnt + kPass - 1) / kPass);
+  const int nch = mp.cols / kChunkCols;
+  d.c0 = (nch * d.ks) / mp.kslices;
+  d.c1 = (nch * (d.ks + 1)) / mp.kslices;
+  d.bsrc = mp.bsrc + static_cast<size_t>(d.prow0) * mp.cols;
+  const pw_block* b = p.pt->blocks + (static_cast<size_t>(p.layer) * p.E + e) * 2 + mode;
+  d.q = b->committed_bits;
+  d.n = b->stored_bits ? b->stored_bits : b->parent_bits;
+  const bool bits_ok = d.q >= b->min_bits && d.q <= d.n && d.n <= b->parent_bits &&
+                       d.q >= PW_MIN_BITS && d.q <= PW_MAX_BITS && b->lut[d.q] != nullptr &&
+                       b->planes != nullptr;
+  const int want_layout = mode == MODE_GATE_UP ? PW_LAYOUT_TILED_GATE_UP : PW_LAYOUT_TILED_DOWN;
+  const bool shape_ok = static_cast<int>(b->rows) == mp.rows &&
+                        static_cast<int>(b->cols) == mp.cols && b->layout == want_layout;
+  const bool resident = b->state == PW_PAGE_GPU;
+  d.tile_words = static_cast<long long>(d.n) * 32 * (mp.cols / 32);
+  // gate_up tiles are 16 gate + 16 up rows (tile index = 16-row group); down tiles 32 rows
+  d.planes = b->planes + static_cast<size_t>(d.mb) * kTiles * d.tile_words;
+  d.lut = bits_ok ? b->lut[d.q] : nullptr;
+  d.valid = bits_ok && shape_ok && resident;
+  d.status = !shape_ok ? PW_ERR_INVALID_ARG : (!resident ? PW_ERR_NOT_RESIDENT : PW_ERR_BAD_BITS);
+  return d;
+}
+
+// ---- tcgen05 wrappers ----
+// Shared-memory matrix descriptor, no swizzle, K-major: start address, leading byte offset
+// (between core matrices adjacent in K), stride byte offset (between 8-row groups), version 1.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3fffu) |
+         (static_cast<uint64_t>((lbo >> 4) & 0x3fffu) << 16) |
+         (static_cast<uint64_t>((sbo >> 4) & 0x3fffu) << 32) | (1ull << 46);
+}
+
+// Instruction descriptor of kind::f16: fp16 A and B (both K-major), fp32 D, M = 128, N = n.
+__device__ __forceinline__ uint32_t instr_desc(int n) {
+  return (1u << 4) | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(kRows >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive (once) on `bar` when every tcgen05.mma this thread issued before has completed.
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::
+                   "r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Generic-proxy writes to shared memory -> visible to the tensor core (async proxy).
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 16 consecutive fp32 columns of this warp's tensor-memory lane quarter, one row per lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  if (*abort_flag) return false;
+  if (!mbar_wait(bar, parity)) {
+    *abort_flag = 1;
+    return false;
+  }
+  return true;
+}
+
+// Every lane of the warp waits; the result is the same in all lanes (false if any lane's
+// wait failed), so no later warp-wide step meets a split warp.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  return __all_sync(0xffffffffu, wait_bar(bar, parity, abort_flag));
+}
+
+using k4::g_smem;
+
+__device__ __forceinline__ uint32_t lds_u32(uint32_t off) {
+  return *reinterpret_cast<const uint32_t*>(g_smem + off);
+}
+
+// One decode warp, one chunk: word wq (32 columns) of tile t's rows at q planes -> 32 fp16
+// weights, stored as four 16-byte core-matrix rows (k-groups 4wq..4wq+3) of the A buffer.
+template <int Q>
+__device__ __forceinline__ void decode_chunk(uint32_t planes_off, uint32_t a_off, int t, int wq,
+                                             int lane) {
+  const int r = t * 32 + lane;  // row of the item's 128
+  // piece (t, p) = [word pair][row][2 words]; this warp's word is (wq / 2, wq % 2)
+  const uint32_t off = planes_off + (wq >> 1) * 256 + lane * 8 + (wq & 1) * 4;
+  uint32_t R[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    R[j] = j < Q ? lds_u32(off + (t * Q + (Q - 1 - j)) * kPieceBytes) : 0u;
+  k4::transpose8(R);  // byte b of R[i] = code of column 8b + i
+  // table address of code v for this row: 512 * (v >> 1) + 4r = ((v & 0xfe) | r >> 6) << 8 |
+  // (4r & 0xff); the byte permute puts the masked code byte in byte 1 of the address
+  const uint32_t rhi = static_cast<uint32_t>(r >> 6) * 0x01010101u;
+  const uint32_t lbase = static_cast<uint32_t>(r * 4) & 0xffu;
+  uint32_t M[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) M[i] = (R[i] & 0xfefefefeu) | rhi;
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    uint32_t w[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const uint32_t sel = 0x7604u | (b << 4);
+      const uint32_t s0 = lds_u32(__byte_perm(M[2 * m], lbase, sel));
+      const uint32_t s1 = lds_u32(__byte_perm(M[2 * m + 1], lbase, sel));
+      // low bits of the two codes -> which half of each slot
+      const uint32_t x = __byte_perm(R[2 * m], R[2 * m + 1], b | ((b + 4) << 4));
+      w[m] = __byte_perm(s0, s1, (x & 0x101u) * 0x22u + 0x5410u);
+    }
+    *reinterpret_cast<uint4*>(g_smem + a_off + (4 * wq + b) * (kRows * 16) + r * 16) =
+        make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// The chunks c0..c1 of one item, one decode warp; returns the chunk counter after them.
+template <int Q>
+__device__ __noinline__ uint32_t decode_item(int c0, int c1, uint64_t* pl_full, uint64_t* pl_empty,
+                                             uint64_t* a_full, uint64_t* ab_empty,
+                                             volatile int* abort_flag, uint32_t g) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = warp & 3, wq = warp >> 2;
+  for (int c = c0; c < c1; ++c, ++g) {
+    const int ps = g % kPlaneStages, ab = g & 1;
+    if (!warp_wait(&pl_full[ps], (g / kPlaneStages) & 1, abort_flag)) return g;
+    if (!warp_wait(&ab_empty[ab], ((g >> 1) & 1) ^ 1, abort_flag)) return g;
+    decode_chunk<Q>(kOffPlanes + ps * kPlaneStageBytes, kOffA + ab * kABytes, t, wq, lane);
+    fence_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(&a_full[ab]);
+      mbar_arrive(&pl_empty[ps]);
+    }
+  }
+  return g;
+}
+
+// Table of tile j's 32 rows for the item: lane = row; slot u of row r at 512u + 4r.
+__device__ __forceinline__ void build_table(const Desc& d, const ModeParams& mp, int j,
+                                            int lane) {
+  const int tile = d.mb * kTiles + j;
+  const int brow = d.mode == MODE_GATE_UP
+                       ? (lane < 16 ? tile * 16 + lane : mp.half + tile * 16 + (lane - 16))
+                       : tile * 32 + lane;
+  const uint4* src = reinterpret_cast<const uint4*>(d.lut + (static_cast<size_t>(brow) << d.q));
+  const int nvec = (1 << d.q) / 8;  // 16-byte pieces of the row (8 entries, 4 slots each)
+  const uint32_t col = (j * 32 + lane) * 4;
+  for (int v0 = 0; v0 < nvec; v0 += 8) {
+    uint4 buf[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (v0 + i < nvec) buf[i] = __ldg(src + v0 + i);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (v0 + i >= nvec) break;
+      const uint32_t u0 = (v0 + i) * 4;
+      *reinterpret_cast<uint32_t*>(g_smem + kOffTable + (u0 + 0) * 512 + col) = buf[i].x;
+      *reinterpret_cast<uint32_t*>(g_smem + kOffTable + (u0 + 1) * 512 + col) = buf[i].y;
+      *reinterpret_cast<uint32_t*>(g_smem + kOffTable + (u0 + 2) * 512 + col) = buf[i].z;
+      *reinterpret_cast<uint32_t*>(g_smem + kOffTable + (u0 + 3) * 512 + col) = buf[i].w;
+    }
+  }
+}
+
+// Epilogue of one item, warp j (rows 32j.. of the accumulator).  gate_up: lanes 0-15 hold the
+// gate rows and lanes 16-31 the matching up rows of features 16 * tile + lane; h = SiLU(gate)
+// * up goes to the down operand staging as fp16, padding tokens included (they are zeros).
+// down: the partial sums of rows 32 * tile + lane for the pass's real tokens.
+__device__ __forceinline__ void epilogue(const Desc& d, const ModeParams& mp, int j, int lane,
+                                         uint32_t tmem_acc) {
+  const int tile = d.mb * kTiles + j;
+  const uint32_t lane_addr = tmem_acc + (static_cast<uint32_t>(j * 32) << 16);
+  for (int c0 = 0; c0 < d.np; c0 += 16) {
+    float v[16];
+    tmem_ld16(lane_addr + c0, v);
+    if (d.mode == MODE_GATE_UP) {
+      const int f = tile * 16 + (lane & 15);
+      // the down operand has I = mp.half columns
+      __half* base = mp.hout + static_cast<size_t>(d.prow0) * mp.half +
+                     (f / 128) * d.np * 128 + ((f % 128) / 8) * d.np * 8 + (f % 8);
+#pragma unroll
+      for (int n = 0; n < 16; ++n) {
+        const float up = __shfl_down_sync(0xffffffffu, v[n], 16);
+        if (lane < 16) {
+          const float g = v[n];
+          base[(c0 + n) * 8] = __float2half_rn(g / (1.0f + expf(-g)) * up);
+        }
+      }
+    } else {
+      float* base = mp.out + d.ks * mp.out_slice + static_cast<size_t>(d.pos0) * mp.ld_out +
+                    tile * 32 + lane;
+#pragma unroll
+      for (int n = 0; n < 16; ++n)
+        if (c0 + n < d.te) base[static_cast<size_t>(c0 + n) * mp.ld_out] = v[n];
+    }
+  }
+}
+
+// Zeros for an item whose block cannot be read (state, bitwidth or shape), warp j.
+__device__ __forceinline__ void zero_outputs(const Desc& d, const ModeParams& mp, int j,
+                                             int lane) {
+  const int tile = d.mb * kTiles + j;
+  if (d.mode == MODE_GATE_UP) {
+    if (lane >= 16) return;
+    const int f = tile * 16 + lane;
+    __half* base = mp.hout + static_cast<size_t>(d.prow0) * mp.half + (f / 128) * d.np * 128 +
+                   ((f % 128) / 8) * d.np * 8 + (f % 8);
+    for (int n = 0; n < d.np; ++n) base[n * 8] = __float2half_rn(0.0f);
+  } else {
+    float* base = mp.out + d.ks * mp.out_slice + static_cast<size_t>(d.pos0) * mp.ld_out +
+                  tile * 32 + lane;
+    for (int n = 0; n < d.te; ++n) base[static_cast<size_t>(n) * mp.ld_out] = 0.0f;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) tc_ffn_kernel(const Params p) {
+  uint8_t* const smem = g_smem;
+  Desc* cdesc = reinterpret_cast<Desc*>(smem + kOffDesc);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* pl_full = bars;
+  uint64_t* pl_empty = pl_full + kPlaneStages;
+  uint64_t* b_full = pl_empty + kPlaneStages;
+  uint64_t* ab_empty = b_full + 2;
+  uint64_t* a_full = ab_empty + 2;
+  uint64_t* acc_full = a_full + 2;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* table_ready = acc_empty + 2;
+  uint64_t* table_free = table_ready + 1;
+  uint64_t* desc_full = table_free + 1;
+  uint64_t* desc_free = desc_full + kDescRing;
+  uint64_t* mma_done = desc_free + kDescRing;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (smem_u32(smem) & 1023) {  // descriptors and buffers assume 1024-byte alignment
+    if (threadIdx.x == 0) set_status(PW_ERR_UNSUPPORTED);
+    return;
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPlaneStages; ++s) {
+      mbar_init(&pl_full[s], 1);
+      mbar_init(&pl_empty[s], kDecodeWarps);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&b_full[b], 1);
+      mbar_init(&ab_empty[b], 1);
+      mbar_init(&a_full[b], kDecodeWarps);
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], kEpiWarps);
+    }
+    mbar_init(table_ready, kEpiWarps);
+    mbar_init(table_free, kDecodeWarps);
+    for (int r = 0; r < kDescRing; ++r) {
+      mbar_init(&desc_full[r], 1);
+      mbar_init(&desc_free[r], 3);  // plane producer, operand producer, MMA
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == kMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  griddep_wait();  // grouping and operand staging of the launches before
+  griddep_launch();
+  const int npass = p.meta[5];
+  const int n_items = items_of(p, MODE_GATE_UP, npass) + items_of(p, MODE_DOWN, npass);
+
+  if (warp == kPlaneWarp) {
+    // ---------------- plane producer ----------------
+    uint32_t g = 0;
+    for (uint32_t j = 0;; ++j) {
+      int stop = 0;
+      if (lane == 0) stop = !wait_bar(&desc_full[j % kDescRing], (j / kDescRing) & 1, abort_flag);
+      stop = __shfl_sync(0xffffffffu, stop, 0);
+      if (stop) break;
+      __syncwarp();  // lane 0's acquire of the descriptor orders the other lanes' reads
+      const Desc d = cdesc[j % kDescRing];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&desc_free[j % kDescRing]);
+      if (d.item < 0) break;
+      if (!d.valid) continue;
+      const int W = p.m[d.mode].cols / 32;
+      for (int c = d.c0; c < d.c1; ++c, ++g) {
+        const int ps = g % kPlaneStages;
+        int ok = 1;
+        if (lane == 0) {
+          ok = wait_bar(&pl_empty[ps], ((g / kPlaneStages) & 1) ^ 1, abort_flag);
+          if (ok) mbar_arrive_expect_tx(&pl_full[ps], kTiles * d.q * kPieceBytes);
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        const int s = c / 8;  // 1024-column stage of the tiled layout
+        const int ws = min(32, W - 32 * s);
+        if (lane < kTiles * d.q) {
+          const int t = lane / d.q, pl = lane - t * d.q;
+          const uint32_t* src = d.planes + t * d.tile_words +
+                                static_cast<size_t>(s) * d.n * 1024 + pl * 32 * ws +
+                                (c % 8) * 128;
+          bulk_g2s(smem + kOffPlanes + ps * kPlaneStageBytes + (t * d.q + pl) * kPieceBytes, src,
+                   kPieceBytes, &pl_full[ps]);
+        }
+        __syncwarp();
+      }
+      if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;
+    }
+    if (lane == 0)  // every issued copy has landed before the block exits
+      for (uint32_t x = (g > kPlaneStages ? g - kPlaneStages : 0); x < g; ++x)
+        mbar_wait(&pl_full[x % kPlaneStages], (x / kPlaneStages) & 1);
+  } else if (warp == kOperandWarp) {
+    // ---------------- operand producer ----------------
+    if (lane == 0) {
+      uint32_t g = 0;
+      for (uint32_t j = 0;; ++j) {
+        if (!wait_bar(&desc_full[j % kDescRing], (j / kDescRing) & 1, abort_flag)) break;
+        const Desc d = cdesc[j % kDescRing];
+        mbar_arrive(&desc_free[j % kDescRing]);
+        if (d.item < 0) break;
+        if (!d.valid) continue;
+        // the down operand (h) of this expert is complete once all its gate_up items count
+        if (d.mode == MODE_DOWN && !k4::wait_count(p.done + d.a, d.target, abort_flag)) break;
+        const uint32_t bytes = d.np * 256;
+        bool ok = true;
+        for (int c = d.c0; c < d.c1; ++c, ++g) {
+          const int b = g & 1;
+          if (!(ok = wait_bar(&ab_empty[b], ((g >> 1) & 1) ^ 1, abort_flag))) break;
+          mbar_arrive_expect_tx(&b_full[b], bytes);
+          bulk_g2s(smem + kOffB + b * kBBytes, d.bsrc + static_cast<size_t>(c) * d.np * 128, bytes,
+                   &b_full[b]);
+        }
+        if (!ok) break;
+      }
+      for (uint32_t x = (g > 2 ? g - 2 : 0); x < g; ++x) mbar_wait(&b_full[x & 1], (x >> 1) & 1);
+    }
+  } else if (warp == kMmaWarp) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      uint32_t g = 0, va = 0;
+      for (uint32_t j = 0;; ++j) {
+        if (!wait_bar(&desc_full[j % kDescRing], (j / kDescRing) & 1, abort_flag)) break;
+        const Desc d = cdesc[j % kDescRing];
+        mbar_arrive(&desc_free[j % kDescRing]);
+        if (d.item < 0) break;
+        if (!d.valid) continue;
+        const uint32_t acc = va & 1;
+        if (!wait_bar(&acc_empty[acc], ((va >> 1) & 1) ^ 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t idesc = instr_desc(d.np);
+        const uint32_t d_tmem = tmem_base + acc * kPass;
+        bool ok = true;
+        for (int c = d.c0; c < d.c1; ++c, ++g) {
+          const int b = g & 1;
+          if (!(ok = wait_bar(&a_full[b], (g >> 1) & 1, abort_flag))) break;
+          if (!(ok = wait_bar(&b_full[b], (g >> 1) & 1, abort_flag))) break;
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + kOffA + b * kABytes);
+          const uint32_t b_addr = smem_u32(smem + kOffB + b * kBBytes);
+#pragma unroll
+          for (int s = 0; s < kChunkCols / 16; ++s)
+            mma_f16(d_tmem, smem_desc(a_addr + s * 2 * kRows * 16, kRows * 16, 128),
+                    smem_desc(b_addr + s * 2 * d.np * 16, d.np * 16, 128), idesc,
+                    (c > d.c0 || s > 0) ? 1u : 0u);
+          mma_commit(&ab_empty[b]);
+        }
+        if (!ok) break;
+        mma_commit(&acc_full[acc]);
+        ++va;
+      }
+      // every issued MMA has completed before the accumulators are released
+      mma_commit(mma_done);
+      mbar_wait(mma_done, 0);
+    }
+  } else if (warp >= kEpiWarp0) {
+    // ---------------- tables, item schedule, epilogue ----------------
+    // The four warps never meet a CTA or named barrier: they follow the descriptors through
+    // their mbarriers, and each counts its own share of a finished gate_up item.
+    const int ew = warp - kEpiWarp0;
+    int item = blockIdx.x;
+    Desc prev;
+    bool have_prev = false;
+    uint32_t va = 0;  // valid items (each fills one accumulator)
+    for (uint32_t j = 0;; ++j) {
+      Desc& slot = cdesc[j % kDescRing];
+      if (ew == 0) {
+        if (lane == 0) {
+          // producers and MMA issuer have read descriptor j - kDescRing from this slot
+          wait_bar(&desc_free[j % kDescRing], ((j / kDescRing) & 1) ^ 1, abort_flag);
+          if (item < n_items && !*abort_flag) {
+            slot = resolve(p, item, npass);
+            slot.item = item;
+            item = gridDim.x + atomicAdd(p.sched, 1);
+          } else {
+            slot.item = -1;
+          }
+          mbar_arrive(&desc_full[j % kDescRing]);
+        }
+        __syncwarp();
+      } else {
+        warp_wait(&desc_full[j % kDescRing], (j / kDescRing) & 1, abort_flag);
+      }
+      const Desc it = slot;
+      // the table is rewritten only after the decode warps left item j - 1
+      const bool freed = warp_wait(table_free, (j & 1) ^ 1, abort_flag);
+      const bool stop = __any_sync(0xffffffffu, it.item < 0 || *abort_flag || !freed);
+      if (!stop && it.valid) build_table(it, p.m[it.mode], ew, lane);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(table_ready);
+      if (stop) break;
+      if (!it.valid) {
+        if (ew == 0 && lane == 0) set_status(it.status);
+        zero_outputs(it, p.m[it.mode], ew, lane);
+        if (it.mode == MODE_GATE_UP) {
+          __threadfence();
+          __syncwarp();
+          if (lane == 0) atomicAdd(p.done + it.a, 1);
+        }
+        continue;
+      }
+      if (have_prev) {
+        // epilogue of the previous valid item while the decode warps work on this one
+        const uint32_t acc = (va - 1) & 1;
+        if (!warp_wait(&acc_full[acc], ((va - 1) >> 1) & 1, abort_flag)) break;
+        tc_fence_after();
+        epilogue(prev, p.m[prev.mode], ew, lane, tmem_base + acc * kPass);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        if (prev.mode == MODE_GATE_UP) {
+          __threadfence();
+          __syncwarp();
+          if (lane == 0) atomicAdd(p.done + prev.a, 1);
+        }
+      }
+      prev = it;
+      have_prev = true;
+      ++va;
+    }
+    if (have_prev) {
+      const uint32_t acc = (va - 1) & 1;
+      if (warp_wait(&acc_full[acc], ((va - 1) >> 1) & 1, abort_flag)) {
+        tc_fence_after();
+        epilogue(prev, p.m[prev.mode], ew, lane, tmem_base + acc * kPass);
+        tc_fence_before();
+        if (prev.mode == MODE_GATE_UP) {
+          __threadfence();
+          __syncwarp();
+          if (lane == 0) atomicAdd(p.done + prev.a, 1);
+        }
+      }
+    }
+  } else {
+    // ---------------- decode warps ----------------
+    uint32_t g = 0;
+    for (uint32_t j = 0;; ++j) {
+      if (!warp_wait(table_ready, j & 1, abort_flag)) break;
+      const Desc d = cdesc[j % kDescRing];
+      if (__any_sync(0xffffffffu, d.item < 0 || *abort_flag)) break;
+      if (d.valid) {
+#define PW_DECODE(Q) decode_item<Q>(d.c0, d.c1, pl_full, pl_empty, a_full, ab_empty, abort_flag, g)
+        switch (d.q) {
+          case 3: g = PW_DECODE(3); break;
+          case 4: g = PW_DECODE(4); break;
+          case 5: g = PW_DECODE(5); break;
+          case 6: g = PW_DECODE(6); break;
+          case 7: g = PW_DECODE(7); break;
+          default: g = PW_DECODE(8); break;
+        }
+#undef PW_DECODE
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(table_free);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+}  // namespace k5
+}  // namespace pw

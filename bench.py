@@ -44,6 +44,8 @@ def parse_args():
     ap.add_argument("--impl", choices=("pw", "reference"), default="pw")
     ap.add_argument("--workload", default=f"{WORKLOAD[0]}:{WORKLOAD[1]}",
                     help="config name:T (default mixtral_8x7b:1)")
+    ap.add_argument("--no-rewrite", action="store_true",
+                    help="plain top-k routing: leave out the config's substitution or remap")
     ap.add_argument("--affinity", action="store_true",
                     help="rewrite the assignments with LYNX AffinityBinning (pw_affinity_remap) "
                          "in place of the config's own rewrite")
@@ -62,11 +64,13 @@ def parse_args():
 
 def workload(args):
     import dataclasses
-    from any_precision_expert_pw_b200.inputs import CONFIGS, POLICY_AFFINITY
+    from any_precision_expert_pw_b200.inputs import CONFIGS, POLICY_AFFINITY, POLICY_NONE
     name, T = args.workload.split(":")
     cfg = CONFIGS[name]
     if getattr(args, "affinity", False):
         cfg = dataclasses.replace(cfg, policy=POLICY_AFFINITY)
+    if getattr(args, "no_rewrite", False):
+        cfg = dataclasses.replace(cfg, policy=POLICY_NONE, resident_frac=None)
     return cfg, int(T)
 
 
