@@ -14,11 +14,13 @@
 //                          words gives one code byte per weight, a gather from the row's table
 //                          gives the fp16 value, and the 32 values go to the chunk's A buffer
 //                          in the MMA's K-major core-matrix order;
-//   table/epilogue (4)     warp 16 + j: builds the decode table of tile j's 32 rows for every
-//                          item, and reads rows 32j.. of the accumulator back (tensor-memory lane
-//                          quarter j) for the epilogue: SiLU(gate) * up as fp16 into the down
-//                          projection's operand, or the down rows into the k-slice partials;
-//                          warp 16 also takes the items (first blockIdx.x, then a work counter);
+//                          At each item's start the sixteen warps first build its decode table
+//                          together (warp w: tile w % 4, a quarter of the slots);
+//   epilogue (4)           warp 16 + j reads rows 32j.. of the accumulator back (tensor-memory
+//                          lane quarter j): SiLU(gate) * up as fp16 into the down projection's
+//                          operand, or the down rows into the k-slice partials; warp 16 also
+//                          takes the items (first blockIdx.x, then a work counter), one ahead,
+//                          and prefetches the next item's LUT rows and first planes into L2;
 //   plane producer (1)     bulk-copies each chunk's top-q planes of the four tiles (4q runs of
 //                          512 bytes in the tiled layout) into a ring of four stages;
 //   operand producer (1)   bulk-copies each chunk's activations (np * 256 contiguous bytes);
@@ -27,8 +29,11 @@
 //   MMA (1)                one thread issues 8 tcgen05.mma (K = 16 each) per chunk into one of
 //                          two accumulators and commits each chunk's completion to the barrier
 //                          that frees its A and B buffers.
-// The decode table holds, for row r, slot u = (LUT[2u], LUT[2u+1]) at byte 512u + 4r, so a
-// warp's gathers hit 32 different banks; the code's low bit picks the half.
+// The decode table pairs rows r and r + 64 of the item: the 32-bit slot at byte 256v + 4r
+// (r < 64) holds (LUT_r[v], LUT_{r+64}[v]).  A warp's 32 rows are 32 consecutive r mod 64, so
+// its gathers hit 32 different banks, the slot address is one byte permute of the code byte,
+// and which half a warp takes is fixed (tiles 0-1 low, 2-3 high): one more byte permute packs
+// two weights.
 #pragma once
 #include "pw_common.cuh"
 #include "pw_ffn.cuh"
@@ -51,9 +56,10 @@ constexpr int kThreads = 23 * 32;
 constexpr int kTmemCols = 2 * kPass;  // two accumulators of up to 64 fp32 columns
 constexpr int kPlaneStages = 4;
 constexpr int kDescRing = 8;
+constexpr int kDescReaders = 3 + kDecodeWarps + 3;
 
 constexpr int kOffTable = 0;
-constexpr int kTableBytes = 128 * kRows * 4;            // 2^8 / 2 slots x 128 rows x 4 bytes
+constexpr int kTableBytes = 256 * 64 * 4;               // 2^8 entries x 64 row pairs x 4 bytes
 constexpr int kOffA = kOffTable + kTableBytes;
 constexpr int kABytes = (kChunkCols / 8) * kRows * 16;  // [16 k-groups][128 rows][16 bytes]
 constexpr int kOffB = kOffA + 2 * kABytes;
@@ -231,8 +237,9 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
   return true;
 }
 
-// Every lane of the warp waits; the result is the same in all lanes (false if any lane's
-// wait failed), so no later warp-wide step meets a split warp.
+// Every lane of the warp waits (a wait by lane 0 alone, the others held at a warp barrier,
+// measured about twice as slow for the decode warps); the result is the same in all lanes
+// (false if any lane's wait failed), so no later warp-wide step meets a split warp.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   return __all_sync(0xffffffffu, wait_bar(bar, parity, abort_flag));
 }
@@ -256,24 +263,18 @@ __device__ __forceinline__ void decode_chunk(uint32_t planes_off, uint32_t a_off
   for (int j = 0; j < 8; ++j)
     R[j] = j < Q ? lds_u32(off + (t * Q + (Q - 1 - j)) * kPieceBytes) : 0u;
   k4::transpose8(R);  // byte b of R[i] = code of column 8b + i
-  // table address of code v for this row: 512 * (v >> 1) + 4r = ((v & 0xfe) | r >> 6) << 8 |
-  // (4r & 0xff); the byte permute puts the masked code byte in byte 1 of the address
-  const uint32_t rhi = static_cast<uint32_t>(r >> 6) * 0x01010101u;
-  const uint32_t lbase = static_cast<uint32_t>(r * 4) & 0xffu;
-  uint32_t M[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) M[i] = (R[i] & 0xfefefefeu) | rhi;
+  // slot address of code v: 256v + 4 (r mod 64); the byte permute puts v in byte 1
+  const uint32_t lbase = static_cast<uint32_t>((r & 63) * 4);
+  const uint32_t psel = (t >> 1) ? 0x7632u : 0x5410u;  // high or low halves
 #pragma unroll
   for (int b = 0; b < 4; ++b) {
     uint32_t w[4];
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
       const uint32_t sel = 0x7604u | (b << 4);
-      const uint32_t s0 = lds_u32(__byte_perm(M[2 * m], lbase, sel));
-      const uint32_t s1 = lds_u32(__byte_perm(M[2 * m + 1], lbase, sel));
-      // low bits of the two codes -> which half of each slot
-      const uint32_t x = __byte_perm(R[2 * m], R[2 * m + 1], b | ((b + 4) << 4));
-      w[m] = __byte_perm(s0, s1, (x & 0x101u) * 0x22u + 0x5410u);
+      const uint32_t s0 = lds_u32(kOffTable + __byte_perm(R[2 * m], lbase, sel));
+      const uint32_t s1 = lds_u32(kOffTable + __byte_perm(R[2 * m + 1], lbase, sel));
+      w[m] = __byte_perm(s0, s1, psel);
     }
     *reinterpret_cast<uint4*>(g_smem + a_off + (4 * wq + b) * (kRows * 16) + r * 16) =
         make_uint4(w[0], w[1], w[2], w[3]);
@@ -302,31 +303,66 @@ __device__ __noinline__ uint32_t decode_item(int c0, int c1, uint64_t* pl_full, 
   return g;
 }
 
-// Table of tile j's 32 rows for the item: lane = row; slot u of row r at 512u + 4r.
-__device__ __forceinline__ void build_table(const Desc& d, const ModeParams& mp, int j,
-                                            int lane) {
-  const int tile = d.mb * kTiles + j;
-  const int brow = d.mode == MODE_GATE_UP
-                       ? (lane < 16 ? tile * 16 + lane : mp.half + tile * 16 + (lane - 16))
-                       : tile * 32 + lane;
-  const uint4* src = reinterpret_cast<const uint4*>(d.lut + (static_cast<size_t>(brow) << d.q));
-  const int nvec = (1 << d.q) / 8;  // 16-byte pieces of the row (8 entries, 4 slots each)
-  const uint32_t col = (j * 32 + lane) * 4;
-  for (int v0 = 0; v0 < nvec; v0 += 8) {
-    uint4 buf[8];
+// LUT row of the block behind row r of the item's 128 (gate_up: rows 16 * tile .. of the gate
+// half for tile rows 0-15, the matching up rows for 16-31).
+__device__ __forceinline__ int block_row(const Desc& d, const ModeParams& mp, int r) {
+  const int tile = d.mb * kTiles + (r >> 5), i = r & 31;
+  if (d.mode == MODE_GATE_UP) return i < 16 ? tile * 16 + i : mp.half + tile * 16 + (i - 16);
+  return tile * 32 + i;
+}
+
+// Decode warp w's share of the item's table: row pair (r, r + 64) with r = 32 (w % 2) + lane,
+// entries [(w / 2) * 2^q / 8, (w / 2 + 1) * 2^q / 8).
+__device__ __forceinline__ void build_part(const Desc& d, const ModeParams& mp, int w, int lane) {
+  const int r = 32 * (w & 1) + lane;
+  const int ne = 1 << (d.q - 3);  // entries of this share
+  const int v0 = (w >> 1) * ne;
+  const uint16_t* lo = d.lut + (static_cast<size_t>(block_row(d, mp, r)) << d.q) + v0;
+  const uint16_t* hi = d.lut + (static_cast<size_t>(block_row(d, mp, r + 64)) << d.q) + v0;
+  uint8_t* dst = g_smem + kOffTable + v0 * 256 + r * 4;
+  if (ne >= 8) {  // 16-byte loads, 8 entries each
+    uint4 a[4], b[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      if (v0 + i < nvec) buf[i] = __ldg(src + v0 + i);
+    for (int i = 0; i < 4; ++i)
+      if (8 * i < ne) {
+        a[i] = __ldg(reinterpret_cast<const uint4*>(lo) + i);
+        b[i] = __ldg(reinterpret_cast<const uint4*>(hi) + i);
+      }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (v0 + i >= nvec) break;
-      const uint32_t u0 = (v0 + i) * 4;
-      *reinterpret_cast<uint32_t*>(g_smem + kOffTable + (u0 + 0) * 512 + col) = buf[i].x;
-      *reinterpret_cast<uint32_t*>(g_smem + kOffTable + (u0 + 1) * 512 + col) = buf[i].y;
-      *reinterpret_cast<uint32_t*>(g_smem + kOffTable + (u0 + 2) * 512 + col) = buf[i].z;
-      *reinterpret_cast<uint32_t*>(g_smem + kOffTable + (u0 + 3) * 512 + col) = buf[i].w;
+    for (int i = 0; i < 4; ++i) {
+      if (8 * i >= ne) break;
+      const uint32_t aw[4] = {a[i].x, a[i].y, a[i].z, a[i].w};
+      const uint32_t bw[4] = {b[i].x, b[i].y, b[i].z, b[i].w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        *reinterpret_cast<uint32_t*>(dst + (8 * i + 2 * k) * 256) = __byte_perm(aw[k], bw[k], 0x5410u);
+        *reinterpret_cast<uint32_t*>(dst + (8 * i + 2 * k + 1) * 256) = __byte_perm(aw[k], bw[k], 0x7632u);
+      }
     }
+  } else {
+    for (int v = 0; v < ne; ++v)
+      *reinterpret_cast<uint32_t*>(dst + v * 256) =
+          static_cast<uint32_t>(__ldg(lo + v)) | (static_cast<uint32_t>(__ldg(hi + v)) << 16);
   }
+}
+
+// L2 prefetch of what an item reads first: the LUT rows of its 128 rows and, for each of its
+// four tiles, the top q planes of its first 1024-column stage.
+__device__ __forceinline__ void prefetch_item(const Params& p, const Desc& d) {
+  if (!d.valid) return;
+  const ModeParams& mp = p.m[d.mode];
+  const uint32_t row_bytes = 2u << d.q;
+  if (d.mode == MODE_GATE_UP) {
+    prefetch_l2(d.lut + (static_cast<size_t>(d.mb * 64) << d.q), 64 * row_bytes);
+    prefetch_l2(d.lut + (static_cast<size_t>(mp.half + d.mb * 64) << d.q), 64 * row_bytes);
+  } else {
+    prefetch_l2(d.lut + (static_cast<size_t>(d.mb * kRows) << d.q), kRows * row_bytes);
+  }
+  const int W = mp.cols / 32, s = d.c0 / 8;
+  const int ws = min(32, W - 32 * s);
+  for (int t = 0; t < kTiles; ++t)
+    prefetch_l2(d.planes + t * d.tile_words + static_cast<size_t>(s) * d.n * 1024,
+                d.q * 32 * ws * 4);
 }
 
 // Epilogue of one item, warp j (rows 32j.. of the accumulator).  gate_up: lanes 0-15 hold the
@@ -416,11 +452,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ffn_kernel(const Params p) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], kEpiWarps);
     }
-    mbar_init(table_ready, kEpiWarps);
+    mbar_init(table_ready, kDecodeWarps);
     mbar_init(table_free, kDecodeWarps);
     for (int r = 0; r < kDescRing; ++r) {
       mbar_init(&desc_full[r], 1);
-      mbar_init(&desc_free[r], 3);  // plane producer, operand producer, MMA
+      // read by: plane and operand producers, MMA issuer, 16 decode warps, epilogue warps 1-3
+      mbar_init(&desc_free[r], kDescReaders);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -548,11 +585,19 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ffn_kernel(const Params p) {
       mbar_wait(mma_done, 0);
     }
   } else if (warp >= kEpiWarp0) {
-    // ---------------- tables, item schedule, epilogue ----------------
+    // ---------------- item schedule, epilogue ----------------
     // The four warps never meet a CTA or named barrier: they follow the descriptors through
     // their mbarriers, and each counts its own share of a finished gate_up item.
     const int ew = warp - kEpiWarp0;
-    int item = blockIdx.x;
+    Desc next;  // warp 16, lane 0: the item claimed for the next descriptor
+    if (ew == 0 && lane == 0) {
+      next.item = -1;
+      if (static_cast<int>(blockIdx.x) < n_items) {
+        next = resolve(p, blockIdx.x, npass);
+        next.item = blockIdx.x;
+        prefetch_item(p, next);
+      }
+    }
     Desc prev;
     bool have_prev = false;
     uint32_t va = 0;  // valid items (each fills one accumulator)
@@ -560,29 +605,31 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ffn_kernel(const Params p) {
       Desc& slot = cdesc[j % kDescRing];
       if (ew == 0) {
         if (lane == 0) {
-          // producers and MMA issuer have read descriptor j - kDescRing from this slot
+          // every reader has read descriptor j - kDescRing from this slot
           wait_bar(&desc_free[j % kDescRing], ((j / kDescRing) & 1) ^ 1, abort_flag);
-          if (item < n_items && !*abort_flag) {
-            slot = resolve(p, item, npass);
-            slot.item = item;
-            item = gridDim.x + atomicAdd(p.sched, 1);
-          } else {
-            slot.item = -1;
-          }
+          if (*abort_flag) next.item = -1;
+          slot = next;
           mbar_arrive(&desc_full[j % kDescRing]);
+          if (next.item >= 0) {
+            const int it2 = gridDim.x + atomicAdd(p.sched, 1);
+            next.item = -1;
+            if (it2 < n_items) {
+              next = resolve(p, it2, npass);
+              next.item = it2;
+              prefetch_item(p, next);
+            }
+          }
         }
         __syncwarp();
       } else {
         warp_wait(&desc_full[j % kDescRing], (j / kDescRing) & 1, abort_flag);
       }
       const Desc it = slot;
-      // the table is rewritten only after the decode warps left item j - 1
-      const bool freed = warp_wait(table_free, (j & 1) ^ 1, abort_flag);
-      const bool stop = __any_sync(0xffffffffu, it.item < 0 || *abort_flag || !freed);
-      if (!stop && it.valid) build_table(it, p.m[it.mode], ew, lane);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(table_ready);
-      if (stop) break;
+      if (ew != 0) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&desc_free[j % kDescRing]);
+      }
+      if (__any_sync(0xffffffffu, it.item < 0 || *abort_flag)) break;
       if (!it.valid) {
         if (ew == 0 && lane == 0) set_status(it.status);
         zero_outputs(it, p.m[it.mode], ew, lane);
@@ -627,25 +674,34 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ffn_kernel(const Params p) {
     }
   } else {
     // ---------------- decode warps ----------------
-    uint32_t g = 0;
+    uint32_t g = 0, vt = 0;
     for (uint32_t j = 0;; ++j) {
-      if (!warp_wait(table_ready, j & 1, abort_flag)) break;
+      if (!warp_wait(&desc_full[j % kDescRing], (j / kDescRing) & 1, abort_flag)) break;
       const Desc d = cdesc[j % kDescRing];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&desc_free[j % kDescRing]);
       if (__any_sync(0xffffffffu, d.item < 0 || *abort_flag)) break;
-      if (d.valid) {
+      if (!d.valid) continue;
+      // the table is rewritten once every decode warp has left the previous item; all sixteen
+      // build it, and decode once all shares are in
+      if (!warp_wait(table_free, (vt & 1) ^ 1, abort_flag)) break;
+      build_part(d, p.m[d.mode], warp, lane);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(table_ready);
+      if (!warp_wait(table_ready, vt & 1, abort_flag)) break;
 #define PW_DECODE(Q) decode_item<Q>(d.c0, d.c1, pl_full, pl_empty, a_full, ab_empty, abort_flag, g)
-        switch (d.q) {
-          case 3: g = PW_DECODE(3); break;
-          case 4: g = PW_DECODE(4); break;
-          case 5: g = PW_DECODE(5); break;
-          case 6: g = PW_DECODE(6); break;
-          case 7: g = PW_DECODE(7); break;
-          default: g = PW_DECODE(8); break;
-        }
-#undef PW_DECODE
+      switch (d.q) {
+        case 3: g = PW_DECODE(3); break;
+        case 4: g = PW_DECODE(4); break;
+        case 5: g = PW_DECODE(5); break;
+        case 6: g = PW_DECODE(6); break;
+        case 7: g = PW_DECODE(7); break;
+        default: g = PW_DECODE(8); break;
       }
+#undef PW_DECODE
       __syncwarp();
       if (lane == 0) mbar_arrive(table_free);
+      ++vt;
     }
   }
 
