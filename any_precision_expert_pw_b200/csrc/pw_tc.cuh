@@ -6,14 +6,16 @@
 //
 // Work item = (active expert, pass of up to 64 of its tokens, 128-row block = four 32-row
 // tiles, k-slice).  D[128 rows][np tokens] (fp32, in tensor memory) += A[128][K] * B[np][K]^T,
-// with A the decoded weights (fp16 LUT values, exact) and B the pass's activations (fp16).
+// with A the decoded weights (fp16 LUT values, exact; in tensor memory) and B the pass's
+// activations (fp16, in shared memory).
 //
 // Warp roles (one CTA per SM, persistent over the items):
 //   decode (16 warps)      warp w takes tile w % 4 of the block and word w / 4 of each
 //                          128-column chunk; lane = row.  An 8x8 bit transpose of its q plane
 //                          words gives one code byte per weight, a gather from the row's table
 //                          gives the fp16 value, and the 32 values go to the chunk's A buffer
-//                          in the MMA's K-major core-matrix order;
+//                          in tensor memory (the warp's own lane quarter, two fp16 per column)
+//                          with one tcgen05.st;
 //                          At each item's start the sixteen warps first build its decode table
 //                          together (warp w: tile w % 4, a quarter of the slots);
 //   epilogue (4)           warp 16 + j reads rows 32j.. of the accumulator back (tensor-memory
@@ -53,16 +55,18 @@ constexpr int kPlaneWarp = 20;
 constexpr int kOperandWarp = 21;
 constexpr int kMmaWarp = 22;
 constexpr int kThreads = 23 * 32;
-constexpr int kTmemCols = 2 * kPass;  // two accumulators of up to 64 fp32 columns
+// tensor memory: two accumulators of up to 64 fp32 columns, then two A buffers of 64 columns
+// (128 rows x 128 fp16)
+constexpr int kTmemCols = 256;
+constexpr int kTmemA = 2 * kPass;
+constexpr int kACols = kChunkCols / 2;
 constexpr int kPlaneStages = 4;
 constexpr int kDescRing = 8;
 constexpr int kDescReaders = 3 + kDecodeWarps + 3;
 
 constexpr int kOffTable = 0;
 constexpr int kTableBytes = 256 * 64 * 4;               // 2^8 entries x 64 row pairs x 4 bytes
-constexpr int kOffA = kOffTable + kTableBytes;
-constexpr int kABytes = (kChunkCols / 8) * kRows * 16;  // [16 k-groups][128 rows][16 bytes]
-constexpr int kOffB = kOffA + 2 * kABytes;
+constexpr int kOffB = kOffTable + kTableBytes;
 constexpr int kBBytes = (kChunkCols / 8) * kPass * 16;  // [16 k-groups][np rows][16 bytes]
 constexpr int kOffPlanes = kOffB + 2 * kBBytes;
 constexpr int kPieceBytes = 512;                        // one plane of one tile for one chunk
@@ -115,7 +119,7 @@ constexpr int kOffBar = kOffDesc + kDescRing * static_cast<int>(sizeof(Desc));
 constexpr int kNumBars = 2 * kPlaneStages + 10 + 2 + 2 * kDescRing + 1;
 constexpr int kSmem = kOffBar + kNumBars * 8 + 16;
 static_assert(kSmem <= 227 * 1024, "shared memory budget");
-static_assert(kOffA % 1024 == 0 && kOffB % 1024 == 0 && kOffPlanes % 1024 == 0, "alignment");
+static_assert(kOffB % 1024 == 0 && kOffPlanes % 1024 == 0, "alignment");
 
 __device__ __forceinline__ int items_of(const Params& p, int mode, int npass) {
   return npass * p.m[mode].mblocks * p.m[mode].kslices;
@@ -194,6 +198,17 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b,
       : "memory");
 }
 
+// The same with A in tensor memory (a_tmem: lane 0, first column of the 128 x 16 slice).
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive (once) on `bar` when every tcgen05.mma this thread issued before has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::
@@ -251,9 +266,9 @@ __device__ __forceinline__ uint32_t lds_u32(uint32_t off) {
 }
 
 // One decode warp, one chunk: word wq (32 columns) of tile t's rows at q planes -> 32 fp16
-// weights, stored as four 16-byte core-matrix rows (k-groups 4wq..4wq+3) of the A buffer.
+// weights, stored to tensor memory at a_taddr (lane = row; column j holds columns 2j, 2j+1).
 template <int Q>
-__device__ __forceinline__ void decode_chunk(uint32_t planes_off, uint32_t a_off, int t, int wq,
+__device__ __forceinline__ void decode_chunk(uint32_t planes_off, uint32_t a_taddr, int t, int wq,
                                              int lane) {
   const int r = t * 32 + lane;  // row of the item's 128
   // piece (t, p) = [word pair][row][2 words]; this warp's word is (wq / 2, wq % 2)
@@ -266,34 +281,45 @@ __device__ __forceinline__ void decode_chunk(uint32_t planes_off, uint32_t a_off
   // slot address of code v: 256v + 4 (r mod 64); the byte permute puts v in byte 1
   const uint32_t lbase = static_cast<uint32_t>((r & 63) * 4);
   const uint32_t psel = (t >> 1) ? 0x7632u : 0x5410u;  // high or low halves
+  uint32_t w[16];  // w[4b + m] = columns 8b + 2m, 8b + 2m + 1
 #pragma unroll
   for (int b = 0; b < 4; ++b) {
-    uint32_t w[4];
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
       const uint32_t sel = 0x7604u | (b << 4);
       const uint32_t s0 = lds_u32(kOffTable + __byte_perm(R[2 * m], lbase, sel));
       const uint32_t s1 = lds_u32(kOffTable + __byte_perm(R[2 * m + 1], lbase, sel));
-      w[m] = __byte_perm(s0, s1, psel);
+      w[4 * b + m] = __byte_perm(s0, s1, psel);
     }
-    *reinterpret_cast<uint4*>(g_smem + a_off + (4 * wq + b) * (kRows * 16) + r * 16) =
-        make_uint4(w[0], w[1], w[2], w[3]);
   }
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(a_taddr),
+      "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]),
+      "r"(w[8]), "r"(w[9]), "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]),
+      "r"(w[15])
+      : "memory");
+  (void)r;
 }
 
 // The chunks c0..c1 of one item, one decode warp; returns the chunk counter after them.
 template <int Q>
 __device__ __noinline__ uint32_t decode_item(int c0, int c1, uint64_t* pl_full, uint64_t* pl_empty,
                                              uint64_t* a_full, uint64_t* ab_empty,
-                                             volatile int* abort_flag, uint32_t g) {
+                                             volatile int* abort_flag, uint32_t g,
+                                             uint32_t tmem_base) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = warp & 3, wq = warp >> 2;
+  // this warp's lane quarter (rows 32t..) and its 16 columns of each A buffer
+  const uint32_t a_lane = tmem_base + (static_cast<uint32_t>(t * 32) << 16) + kTmemA + 16 * wq;
   for (int c = c0; c < c1; ++c, ++g) {
     const int ps = g % kPlaneStages, ab = g & 1;
     if (!warp_wait(&pl_full[ps], (g / kPlaneStages) & 1, abort_flag)) return g;
     if (!warp_wait(&ab_empty[ab], ((g >> 1) & 1) ^ 1, abort_flag)) return g;
-    decode_chunk<Q>(kOffPlanes + ps * kPlaneStageBytes, kOffA + ab * kABytes, t, wq, lane);
-    fence_async_smem();
+    tc_fence_after();  // the MMA that read this A buffer has completed
+    decode_chunk<Q>(kOffPlanes + ps * kPlaneStageBytes, a_lane + ab * kACols, t, wq, lane);
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+    tc_fence_before();
     __syncwarp();
     if (lane == 0) {
       mbar_arrive(&a_full[ab]);
@@ -567,13 +593,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ffn_kernel(const Params p) {
           if (!(ok = wait_bar(&a_full[b], (g >> 1) & 1, abort_flag))) break;
           if (!(ok = wait_bar(&b_full[b], (g >> 1) & 1, abort_flag))) break;
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem + kOffA + b * kABytes);
+          const uint32_t a_tmem = tmem_base + kTmemA + b * kACols;
           const uint32_t b_addr = smem_u32(smem + kOffB + b * kBBytes);
 #pragma unroll
-          for (int s = 0; s < kChunkCols / 16; ++s)
-            mma_f16(d_tmem, smem_desc(a_addr + s * 2 * kRows * 16, kRows * 16, 128),
-                    smem_desc(b_addr + s * 2 * d.np * 16, d.np * 16, 128), idesc,
-                    (c > d.c0 || s > 0) ? 1u : 0u);
+          for (int s = 0; s < kChunkCols / 16; ++s)  // K = 16: 8 columns of A
+            mma_f16_ts(d_tmem, a_tmem + 8 * s, smem_desc(b_addr + s * 2 * d.np * 16, d.np * 16, 128),
+                       idesc, (c > d.c0 || s > 0) ? 1u : 0u);
           mma_commit(&ab_empty[b]);
         }
         if (!ok) break;
@@ -689,7 +714,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ffn_kernel(const Params p) {
       __syncwarp();
       if (lane == 0) mbar_arrive(table_ready);
       if (!warp_wait(table_ready, vt & 1, abort_flag)) break;
-#define PW_DECODE(Q) decode_item<Q>(d.c0, d.c1, pl_full, pl_empty, a_full, ab_empty, abort_flag, g)
+#define PW_DECODE(Q) \
+  decode_item<Q>(d.c0, d.c1, pl_full, pl_empty, a_full, ab_empty, abort_flag, g, tmem_base)
       switch (d.q) {
         case 3: g = PW_DECODE(3); break;
         case 4: g = PW_DECODE(4); break;
