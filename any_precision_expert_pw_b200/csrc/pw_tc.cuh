@@ -729,6 +729,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ffn_kernel(const Params p) {
       if (lane == 0) mbar_arrive(table_free);
       ++vt;
     }
+    // an item left early (abort) may have a store in flight: it lands before the release
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
   }
 
   tc_fence_before();
