@@ -85,7 +85,7 @@ def read_peaks():
 
 
 # the sources of the kernels pw_moe_anyprec_forward launches (and their launch logic)
-FORWARD_SOURCES = ("pw_common.cuh", "pw_ffn.cuh", "pw_group.cuh", "pw_lib.cu")
+FORWARD_SOURCES = ("pw_common.cuh", "pw_ffn.cuh", "pw_group.cuh", "pw_lib.cu", "pw_tc.cuh")
 
 
 def kernel_source_hash():
@@ -97,8 +97,9 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
-def recorded_traffic():
-    """DRAM traffic per FFN call from the committed ncu summary, if it matches this source."""
+def recorded_traffic(workload_key: str):
+    """DRAM traffic per FFN call from the committed ncu summary, if it was taken on this
+    workload (`name:T`, default routing) with these sources."""
     p = os.path.join(ROOT, "profiles", "ffn_traffic.txt")
     try:
         kv = {}
@@ -106,7 +107,7 @@ def recorded_traffic():
             if "=" in line and not line.startswith("#"):
                 k, v = line.strip().split("=", 1)
                 kv[k.strip()] = v.strip()
-        if kv.get("source_sha") == kernel_source_hash():
+        if kv.get("source_sha") == kernel_source_hash() and kv.get("workload") == workload_key:
             return float(kv["traffic_bytes_per_call"])
     except Exception:
         pass
@@ -413,7 +414,8 @@ def run_pw(args):
     b_planes = plane_bytes(cfg.H, cfg.I, L.q, used)
     peak, peak_kind = read_peaks()
     achieved = b_ffn / (ffn_ms * 1e-3) / 1e9
-    traffic = recorded_traffic()
+    plain = not (getattr(args, "affinity", False) or getattr(args, "no_rewrite", False))
+    traffic = recorded_traffic(f"{cfg.name}:{T}") if plain else None
     value = replica_value(world, T, step_ms)
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
