@@ -335,7 +335,11 @@ def run_pw(args):
         D.ffn()
     # router (+ top-k, fused into it when the E experts fit one CTA of 8), the assignment
     # rewrite if any, then setup, the FFN (gate_up and down in one launch) and combine
-    launches_step = (1 if cfg.E <= 8 else 2) + (0 if cfg.policy == POLICY_NONE else 1) + 3
+    # router (+ separate top-k for E > 8), rewrite, setup, FFN, combine; the tensor-core FFN
+    # (taken at >= 8 routed tokens per active expert, the library default) adds its staging
+    tc_path = T * cfg.k >= 8 * min(cfg.E, T * cfg.k)
+    launches_step = ((1 if cfg.E <= 8 else 2) + (0 if cfg.policy == POLICY_NONE else 1) + 3 +
+                     (1 if tc_path else 0))
 
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(int(2.5 * l2), dtype=torch.uint8, device=dev)
