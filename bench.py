@@ -44,6 +44,10 @@ def parse_args():
     ap.add_argument("--impl", choices=("pw", "reference"), default="pw")
     ap.add_argument("--workload", default=f"{WORKLOAD[0]}:{WORKLOAD[1]}",
                     help="config name:T (default mixtral_8x7b:1)")
+    ap.add_argument("--tc-min-tokens", type=int, default=None, metavar="M",
+                    help="switch of the forward call's FFN paths (pw_set_tc_min_tokens): the "
+                         "tensor-core FFN from an average of M routed tokens per active expert "
+                         "(library default 8; 0 = always)")
     ap.add_argument("--no-rewrite", action="store_true",
                     help="plain top-k routing: leave out the config's substitution or remap")
     ap.add_argument("--affinity", action="store_true",
@@ -309,6 +313,8 @@ def run_pw(args):
     dev = torch.device(f"cuda:{local}")
     torch.cuda.set_device(dev)
     cfg, T = workload(args)
+    tc_min = 8 if args.tc_min_tokens is None else args.tc_min_tokens
+    B.check(B.pw_set_tc_min_tokens(tc_min))
     L = make_layer(cfg, T)
     D = DeviceLayer(L, device=str(dev))
     stream = torch.cuda.Stream(device=dev)
@@ -333,11 +339,9 @@ def run_pw(args):
     g_ffn = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_ffn, stream=stream):
         D.ffn()
-    # router (+ top-k, fused into it when the E experts fit one CTA of 8), the assignment
-    # rewrite if any, then setup, the FFN (gate_up and down in one launch) and combine
-    # router (+ separate top-k for E > 8), rewrite, setup, FFN, combine; the tensor-core FFN
-    # (taken at >= 8 routed tokens per active expert, the library default) adds its staging
-    tc_path = T * cfg.k >= 8 * min(cfg.E, T * cfg.k)
+    # router (+ separate top-k for E > 8), the assignment rewrite if any, setup, the FFN
+    # (gate_up and down in one launch) and combine; the tensor-core FFN adds its operand staging
+    tc_path = T * cfg.k >= tc_min * min(cfg.E, T * cfg.k)
     launches_step = ((1 if cfg.E <= 8 else 2) + (0 if cfg.policy == POLICY_NONE else 1) + 3 +
                      (1 if tc_path else 0))
 
@@ -429,6 +433,7 @@ def run_pw(args):
         "config": {"workload": f"{cfg.name}-shaped MoE decode layer, T={T}", "H": cfg.H,
                    "E": cfg.E, "I": cfg.I, "k": cfg.k, "parent_bits": cfg.n,
                    "bits": L.q.tolist(), "experts_used": used.tolist(),
+                   "ffn_path": "tensor-core (tcgen05)" if tc_path else "cuda-core",
                    "rewrite": {-1: "none", 0: "fetch-all", 1: "0.15 rule", 2: "first choice",
                                3: "batch remap", 4: "AffinityBinning remap"}[cfg.policy],
                    "parallelism": f"replicas{world}" if world > 1 else "single",
