@@ -126,7 +126,7 @@ std::mutex g_static_ws_mu;
 
 
 // Average routed tokens per active expert from which the tensor-core FFN is used.
-std::atomic<int> g_tc_min_tokens{8};
+std::atomic<int> g_tc_min_tokens{4};
 
 // k-slices for the down projection: fill the GPU in whole waves of work items, with at least
 // two 1024-column stages per slice.

@@ -47,7 +47,7 @@ def parse_args():
     ap.add_argument("--tc-min-tokens", type=int, default=None, metavar="M",
                     help="switch of the forward call's FFN paths (pw_set_tc_min_tokens): the "
                          "tensor-core FFN from an average of M routed tokens per active expert "
-                         "(library default 8; 0 = always)")
+                         "(library default 4; 0 = always)")
     ap.add_argument("--no-rewrite", action="store_true",
                     help="plain top-k routing: leave out the config's substitution or remap")
     ap.add_argument("--affinity", action="store_true",
@@ -313,7 +313,7 @@ def run_pw(args):
     dev = torch.device(f"cuda:{local}")
     torch.cuda.set_device(dev)
     cfg, T = workload(args)
-    tc_min = 8 if args.tc_min_tokens is None else args.tc_min_tokens
+    tc_min = 4 if args.tc_min_tokens is None else args.tc_min_tokens
     B.check(B.pw_set_tc_min_tokens(tc_min))
     L = make_layer(cfg, T)
     D = DeviceLayer(L, device=str(dev))

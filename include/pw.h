@@ -291,7 +291,7 @@ size_t pw_moe_workspace_bytes(int T, int k, int E, int H, int I);
  *   contribution is zero).  H % 128 == 0, I % 128 == 0.
  *   Two FFN paths give the same result within the tolerance of the arithmetic (the choice
  *   never changes routing): while T*k < m * min(E, T*k) (m = pw_set_tc_min_tokens, default
- *   8) a CUDA-core bit-plane GEMV in fp32 (each weight decoded once per four tokens);
+ *   4) a CUDA-core bit-plane GEMV in fp32 (each weight decoded once per four tokens);
  *   otherwise the tensor-core GEMM (tcgen05, fp16 operands, fp32 accumulation; each weight
  *   decoded once per 64 tokens of its expert).  On the tensor-core path the activations are
  *   rounded to fp16 (exact for bf16 values within fp16's normal range) and so is h = SiLU(g)
@@ -330,7 +330,7 @@ pw_status pw_moe_anyprec_forward_static(const pw_page_table* pt_dev, int layer, 
  * pw_set_tc_min_tokens: process-wide switch between the two FFN paths of
  * pw_moe_anyprec_forward: the tensor-core path is taken when the batch routes on average at
  * least `tokens_per_expert` tokens to each active expert (T*k >= m * min(E, T*k)); 0 selects
- * it always, a value above PW_MAX_TOKENS * PW_MAX_TOPK never.  Default 8.  Affects calls
+ * it always, a value above PW_MAX_TOKENS * PW_MAX_TOPK never.  Default 4.  Affects calls
  * made (or graphs captured) after it returns.  PW_ERR_INVALID_ARG for a negative value.
  * ------------------------------------------------------------------------------------- */
 pw_status pw_set_tc_min_tokens(int tokens_per_expert);

@@ -16,7 +16,7 @@ from oracle import layer as olayer
 
 pytestmark = pytest.mark.gpu
 
-DEFAULT_MIN_TOKENS = 8
+DEFAULT_MIN_TOKENS = 4
 
 
 @pytest.fixture
