@@ -11,6 +11,7 @@ namespace pw {
 constexpr int kGroupThreads = 1024;
 constexpr int kMaxAssign = 8192;  // T * k handled by the single-CTA grouping step
 constexpr int kPassTokens = 64;   // tokens of one expert per tensor-core pass (MMA N <= 64)
+constexpr int kTcChunkCols = 256; // K columns per tensor-core pipeline step (operand chunk)
 
 // What the tensor-core FFN needs beyond the plain grouping.  Each expert's tokens are split
 // into passes of up to kPassTokens; a pass of m tokens is padded to np = m rounded up to 16
@@ -178,10 +179,11 @@ __global__ void __launch_bounds__(kGroupThreads) setup_kernel(
 }
 
 // The tensor-core FFN's gate_up operand: for every padded row (ptok, pnn as in PassOut) the
-// token's activations as fp16, in the MMA's K-major core-matrix order per 128-column chunk:
+// token's activations as fp16, in the MMA's K-major core-matrix order per 256-column chunk:
 // element (n, c) of the pass starting at padded row r0 (np rows) sits at
-//   r0 * H + (c / 128) * np * 128 + ((c % 128) / 8) * np * 8 + n * 8 + c % 8
-// (so one chunk of a pass is np * 256 contiguous bytes); padding rows are zeros.  bf16 -> fp16
+//   r0 * H + (c / 256) * np * 256 + ((c % 256) / 8) * np * 8 + n * 8 + c % 8
+// (so one chunk of a pass is np * 512 contiguous bytes, a last chunk of 128 columns half
+// that); padding rows are zeros.  bf16 -> fp16
 // is exact for values in fp16's normal range.  `vec`: x is 16-byte aligned.
 __global__ void __launch_bounds__(256) stage_x_kernel(const uint16_t* __restrict__ x, int H,
                                                       int vec, const int32_t* __restrict__ ptok,
@@ -200,8 +202,8 @@ __global__ void __launch_bounds__(256) stage_x_kernel(const uint16_t* __restrict
     const int tok = ptok[row];
     const int nn = pnn[row];
     const int np = nn >> 16, n = nn & 0xffff;
-    __half* dst = XB + static_cast<size_t>(row - n) * H + (c / 128) * np * 128 +
-                  ((c % 128) / 8) * np * 8 + n * 8;
+    __half* dst = XB + static_cast<size_t>(row - n) * H + (c / kTcChunkCols) * np * kTcChunkCols +
+                  ((c % kTcChunkCols) / 8) * np * 8 + n * 8;
     uint4 out = make_uint4(0u, 0u, 0u, 0u);
     if (tok >= 0) {
       const uint16_t* src = x + static_cast<size_t>(tok) * H + c;

@@ -5,17 +5,17 @@
 // tokens and the products run on tcgen05.
 //
 // Work item = (active expert, pass of up to 64 of its tokens, 128-row block = four 32-row
-// tiles, k-slice).  D[128 rows][np tokens] (fp32, in tensor memory) += A[128][K] * B[np][K]^T,
+// tiles, k-slice).  A block whose columns are not a multiple of 256 ends in a 128-column chunk.  D[128 rows][np tokens] (fp32, in tensor memory) += A[128][K] * B[np][K]^T,
 // with A the decoded weights (fp16 LUT values, exact; in tensor memory) and B the pass's
 // activations (fp16, in shared memory).
 //
 // Warp roles (one CTA per SM, persistent over the items):
-//   decode (16 warps)      warp w takes tile w % 4 of the block and word w / 4 of each
-//                          128-column chunk; lane = row.  An 8x8 bit transpose of its q plane
-//                          words gives one code byte per weight, a gather from the row's table
-//                          gives the fp16 value, and the 32 values go to the chunk's A buffer
-//                          in tensor memory (the warp's own lane quarter, two fp16 per column)
-//                          with one tcgen05.st;
+//   decode (16 warps)      warp w takes tile w % 4 of the block and words 2(w / 4), 2(w / 4) + 1
+//                          (64 columns) of each 256-column chunk; lane = row.  An 8x8 bit
+//                          transpose of its q plane words gives one code byte per weight, a
+//                          gather from the row's table gives the fp16 value, and each word's
+//                          32 values go to the chunk's A buffer in tensor memory (the warp's
+//                          own lane quarter, two fp16 per column) with one tcgen05.st;
 //                          At each item's start the sixteen warps first build its decode table
 //                          together (warp w: tile w % 4, a quarter of the slots);
 //   epilogue (4)           warp 16 + j reads rows 32j.. of the accumulator back (tensor-memory
@@ -24,11 +24,11 @@
 //                          takes the items (first blockIdx.x, then a work counter), one ahead,
 //                          and prefetches the next item's LUT rows and first planes into L2;
 //   plane producer (1)     bulk-copies each chunk's top-q planes of the four tiles (4q runs of
-//                          512 bytes in the tiled layout) into a ring of four stages;
-//   operand producer (1)   bulk-copies each chunk's activations (np * 256 contiguous bytes);
+//                          1 KB in the tiled layout) into a ring of three stages;
+//   operand producer (1)   bulk-copies each chunk's activations (np * 512 contiguous bytes);
 //                          a down item first waits until every gate_up item of its expert is
 //                          counted;
-//   MMA (1)                one thread issues 8 tcgen05.mma (K = 16 each) per chunk into one of
+//   MMA (1)                one thread issues 16 tcgen05.mma (K = 16 each) per chunk into one of
 //                          two accumulators and commits each chunk's completion to the barrier
 //                          that frees its A and B buffers.
 // The decode table pairs rows r and r + 64 of the item: the 32-bit slot at byte 256v + 4r
@@ -46,7 +46,8 @@ namespace k5 {
 
 constexpr int kRows = 128;        // MMA M
 constexpr int kTiles = 4;         // 32-row tiles per item
-constexpr int kChunkCols = 128;   // K columns per pipeline step
+constexpr int kChunkCols = kTcChunkCols;  // K columns per pipeline step (256)
+constexpr int kChunkWords = kChunkCols / 32;
 constexpr int kPass = kPassTokens;
 constexpr int kDecodeWarps = 16;
 constexpr int kEpiWarp0 = 16;
@@ -57,19 +58,19 @@ constexpr int kMmaWarp = 22;
 constexpr int kThreads = 23 * 32;
 // tensor memory: two accumulators of up to 64 fp32 columns, then two A buffers of 64 columns
 // (128 rows x 128 fp16)
-constexpr int kTmemCols = 256;
+constexpr int kTmemCols = 512;  // 128 accumulator + 2 x 128 A columns used
 constexpr int kTmemA = 2 * kPass;
 constexpr int kACols = kChunkCols / 2;
-constexpr int kPlaneStages = 4;
+constexpr int kPlaneStages = 3;
 constexpr int kDescRing = 8;
 constexpr int kDescReaders = 3 + kDecodeWarps + 3;
 
 constexpr int kOffTable = 0;
 constexpr int kTableBytes = 256 * 64 * 4;               // 2^8 entries x 64 row pairs x 4 bytes
 constexpr int kOffB = kOffTable + kTableBytes;
-constexpr int kBBytes = (kChunkCols / 8) * kPass * 16;  // [16 k-groups][np rows][16 bytes]
+constexpr int kBBytes = (kChunkCols / 8) * kPass * 16;  // [32 k-groups][np rows][16 bytes]
 constexpr int kOffPlanes = kOffB + 2 * kBBytes;
-constexpr int kPieceBytes = 512;                        // one plane of one tile for one chunk
+constexpr int kPieceBytes = kChunkWords * 32 * 4;       // one plane of one tile for one chunk
 constexpr int kPlaneStageBytes = kTiles * PW_MAX_BITS * kPieceBytes;
 constexpr int kOffDesc = kOffPlanes + kPlaneStages * kPlaneStageBytes;
 
@@ -151,7 +152,7 @@ __device__ __forceinline__ Desc resolve(const Params& p, int item, int npass) {
   d.prow0 = p.pbase[e] + kPass * j;
   // each of the four epilogue warps counts every gate_up item of the expert once
   d.target = kEpiWarps * p.m[MODE_GATE_UP].mblocks * ((cnt + kPass - 1) / kPass);
-  const int nch = mp.cols / kChunkCols;
+  const int nch = (mp.cols + kChunkCols - 1) / kChunkCols;  // a last chunk may hold 128 columns
   d.c0 = (nch * d.ks) / mp.kslices;
   d.c1 = (nch * (d.ks + 1)) / mp.kslices;
   d.bsrc = mp.bsrc + static_cast<size_t>(d.prow0) * mp.cols;
@@ -265,59 +266,69 @@ __device__ __forceinline__ uint32_t lds_u32(uint32_t off) {
   return *reinterpret_cast<const uint32_t*>(g_smem + off);
 }
 
-// One decode warp, one chunk: word wq (32 columns) of tile t's rows at q planes -> 32 fp16
-// weights, stored to tensor memory at a_taddr (lane = row; column j holds columns 2j, 2j+1).
+// One decode warp, one chunk: words 2jj and 2jj + 1 (64 columns) of tile t's rows at q planes
+// -> 2 x 32 fp16 weights, stored to tensor memory at a_taddr and a_taddr + 16 (lane = row;
+// column j holds columns 2j, 2j + 1 of the pair).
 template <int Q>
-__device__ __forceinline__ void decode_chunk(uint32_t planes_off, uint32_t a_taddr, int t, int wq,
-                                             int lane) {
+__device__ __forceinline__ void decode_pair(uint32_t planes_off, uint32_t a_taddr, int t, int jj,
+                                            int lane) {
   const int r = t * 32 + lane;  // row of the item's 128
-  // piece (t, p) = [word pair][row][2 words]; this warp's word is (wq / 2, wq % 2)
-  const uint32_t off = planes_off + (wq >> 1) * 256 + lane * 8 + (wq & 1) * 4;
-  uint32_t R[8];
+  // piece (t, p) = [word pair][row][2 words]: this warp's pair is 8 bytes per lane
+  const uint32_t off = planes_off + jj * 256 + lane * 8;
+  uint2 P[Q];
 #pragma unroll
-  for (int j = 0; j < 8; ++j)
-    R[j] = j < Q ? lds_u32(off + (t * Q + (Q - 1 - j)) * kPieceBytes) : 0u;
-  k4::transpose8(R);  // byte b of R[i] = code of column 8b + i
+  for (int p = 0; p < Q; ++p)
+    P[p] = *reinterpret_cast<const uint2*>(g_smem + off + (t * Q + p) * kPieceBytes);
   // slot address of code v: 256v + 4 (r mod 64); the byte permute puts v in byte 1
   const uint32_t lbase = static_cast<uint32_t>((r & 63) * 4);
   const uint32_t psel = (t >> 1) ? 0x7632u : 0x5410u;  // high or low halves
-  uint32_t w[16];  // w[4b + m] = columns 8b + 2m, 8b + 2m + 1
 #pragma unroll
-  for (int b = 0; b < 4; ++b) {
+  for (int wi = 0; wi < 2; ++wi) {
+    uint32_t R[8];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const uint32_t sel = 0x7604u | (b << 4);
-      const uint32_t s0 = lds_u32(kOffTable + __byte_perm(R[2 * m], lbase, sel));
-      const uint32_t s1 = lds_u32(kOffTable + __byte_perm(R[2 * m + 1], lbase, sel));
-      w[4 * b + m] = __byte_perm(s0, s1, psel);
+    for (int j = 0; j < 8; ++j) R[j] = j < Q ? (wi ? P[Q - 1 - j].y : P[Q - 1 - j].x) : 0u;
+    k4::transpose8(R);  // byte b of R[i] = code of column 8b + i
+    uint32_t w[16];     // w[4b + m] = columns 8b + 2m, 8b + 2m + 1
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const uint32_t sel = 0x7604u | (b << 4);
+        const uint32_t s0 = lds_u32(kOffTable + __byte_perm(R[2 * m], lbase, sel));
+        const uint32_t s1 = lds_u32(kOffTable + __byte_perm(R[2 * m + 1], lbase, sel));
+        w[4 * b + m] = __byte_perm(s0, s1, psel);
+      }
     }
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(
+            a_taddr + 16 * wi),
+        "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]),
+        "r"(w[8]), "r"(w[9]), "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]),
+        "r"(w[15])
+        : "memory");
   }
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(a_taddr),
-      "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]),
-      "r"(w[8]), "r"(w[9]), "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]),
-      "r"(w[15])
-      : "memory");
-  (void)r;
 }
 
 // The chunks c0..c1 of one item, one decode warp; returns the chunk counter after them.
+// words_total = the block's columns / 32 (a last chunk may hold only 4 words: warps whose pair
+// lies beyond it only take part in the hand-offs).
 template <int Q>
-__device__ __noinline__ uint32_t decode_item(int c0, int c1, uint64_t* pl_full, uint64_t* pl_empty,
-                                             uint64_t* a_full, uint64_t* ab_empty,
-                                             volatile int* abort_flag, uint32_t g,
-                                             uint32_t tmem_base) {
+__device__ __noinline__ uint32_t decode_item(int c0, int c1, int words_total, uint64_t* pl_full,
+                                             uint64_t* pl_empty, uint64_t* a_full,
+                                             uint64_t* ab_empty, volatile int* abort_flag,
+                                             uint32_t g, uint32_t tmem_base) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = warp & 3, wq = warp >> 2;
-  // this warp's lane quarter (rows 32t..) and its 16 columns of each A buffer
-  const uint32_t a_lane = tmem_base + (static_cast<uint32_t>(t * 32) << 16) + kTmemA + 16 * wq;
+  const int t = warp & 3, jj = warp >> 2;
+  // this warp's lane quarter (rows 32t..) and its 32 columns of each A buffer
+  const uint32_t a_lane = tmem_base + (static_cast<uint32_t>(t * 32) << 16) + kTmemA + 32 * jj;
   for (int c = c0; c < c1; ++c, ++g) {
     const int ps = g % kPlaneStages, ab = g & 1;
     if (!warp_wait(&pl_full[ps], (g / kPlaneStages) & 1, abort_flag)) return g;
     if (!warp_wait(&ab_empty[ab], ((g >> 1) & 1) ^ 1, abort_flag)) return g;
     tc_fence_after();  // the MMA that read this A buffer has completed
-    decode_chunk<Q>(kOffPlanes + ps * kPlaneStageBytes, a_lane + ab * kACols, t, wq, lane);
+    if (2 * jj < words_total - kChunkWords * c)
+      decode_pair<Q>(kOffPlanes + ps * kPlaneStageBytes, a_lane + ab * kACols, t, jj, lane);
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
     tc_fence_before();
     __syncwarp();
@@ -384,7 +395,7 @@ __device__ __forceinline__ void prefetch_item(const Params& p, const Desc& d) {
   } else {
     prefetch_l2(d.lut + (static_cast<size_t>(d.mb * kRows) << d.q), kRows * row_bytes);
   }
-  const int W = mp.cols / 32, s = d.c0 / 8;
+  const int W = mp.cols / 32, s = d.c0 * kChunkCols / 1024;
   const int ws = min(32, W - 32 * s);
   for (int t = 0; t < kTiles; ++t)
     prefetch_l2(d.planes + t * d.tile_words + static_cast<size_t>(s) * d.n * 1024,
@@ -406,7 +417,8 @@ __device__ __forceinline__ void epilogue(const Desc& d, const ModeParams& mp, in
       const int f = tile * 16 + (lane & 15);
       // the down operand has I = mp.half columns
       __half* base = mp.hout + static_cast<size_t>(d.prow0) * mp.half +
-                     (f / 128) * d.np * 128 + ((f % 128) / 8) * d.np * 8 + (f % 8);
+                     (f / kChunkCols) * d.np * kChunkCols + ((f % kChunkCols) / 8) * d.np * 8 +
+                     (f % 8);
 #pragma unroll
       for (int n = 0; n < 16; ++n) {
         const float up = __shfl_down_sync(0xffffffffu, v[n], 16);
@@ -432,8 +444,8 @@ __device__ __forceinline__ void zero_outputs(const Desc& d, const ModeParams& mp
   if (d.mode == MODE_GATE_UP) {
     if (lane >= 16) return;
     const int f = tile * 16 + lane;
-    __half* base = mp.hout + static_cast<size_t>(d.prow0) * mp.half + (f / 128) * d.np * 128 +
-                   ((f % 128) / 8) * d.np * 8 + (f % 8);
+    __half* base = mp.hout + static_cast<size_t>(d.prow0) * mp.half +
+                   (f / kChunkCols) * d.np * kChunkCols + ((f % kChunkCols) / 8) * d.np * 8 + (f % 8);
     for (int n = 0; n < d.np; ++n) base[n * 8] = __float2half_rn(0.0f);
   } else {
     float* base = mp.out + d.ks * mp.out_slice + static_cast<size_t>(d.pos0) * mp.ld_out +
@@ -526,19 +538,21 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ffn_kernel(const Params p) {
         int ok = 1;
         if (lane == 0) {
           ok = wait_bar(&pl_empty[ps], ((g / kPlaneStages) & 1) ^ 1, abort_flag);
-          if (ok) mbar_arrive_expect_tx(&pl_full[ps], kTiles * d.q * kPieceBytes);
+          if (ok)
+            mbar_arrive_expect_tx(&pl_full[ps],
+                                  kTiles * d.q * min(kChunkWords, W - kChunkWords * c) * 128);
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
-        const int s = c / 8;  // 1024-column stage of the tiled layout
+        const int s = c / 4;  // 1024-column stage of the tiled layout
         const int ws = min(32, W - 32 * s);
         if (lane < kTiles * d.q) {
           const int t = lane / d.q, pl = lane - t * d.q;
           const uint32_t* src = d.planes + t * d.tile_words +
                                 static_cast<size_t>(s) * d.n * 1024 + pl * 32 * ws +
-                                (c % 8) * 128;
+                                (c % 4) * kChunkWords * 32;
           bulk_g2s(smem + kOffPlanes + ps * kPlaneStageBytes + (t * d.q + pl) * kPieceBytes, src,
-                   kPieceBytes, &pl_full[ps]);
+                   min(kChunkWords, W - kChunkWords * c) * 128, &pl_full[ps]);
         }
         __syncwarp();
       }
@@ -559,14 +573,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ffn_kernel(const Params p) {
         if (!d.valid) continue;
         // the down operand (h) of this expert is complete once all its gate_up items count
         if (d.mode == MODE_DOWN && !k4::wait_count(p.done + d.a, d.target, abort_flag)) break;
-        const uint32_t bytes = d.np * 256;
+        const int W = p.m[d.mode].cols / 32;
         bool ok = true;
         for (int c = d.c0; c < d.c1; ++c, ++g) {
           const int b = g & 1;
+          // np rows x the chunk's columns (256, or 128 for a last half chunk) of fp16
+          const uint32_t bytes = d.np * min(kChunkWords, W - kChunkWords * c) * 64;
           if (!(ok = wait_bar(&ab_empty[b], ((g >> 1) & 1) ^ 1, abort_flag))) break;
           mbar_arrive_expect_tx(&b_full[b], bytes);
-          bulk_g2s(smem + kOffB + b * kBBytes, d.bsrc + static_cast<size_t>(c) * d.np * 128, bytes,
-                   &b_full[b]);
+          bulk_g2s(smem + kOffB + b * kBBytes,
+                   d.bsrc + static_cast<size_t>(c) * d.np * kChunkCols, bytes, &b_full[b]);
         }
         if (!ok) break;
       }
@@ -587,6 +603,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ffn_kernel(const Params p) {
         tc_fence_after();
         const uint32_t idesc = instr_desc(d.np);
         const uint32_t d_tmem = tmem_base + acc * kPass;
+        const int W = p.m[d.mode].cols / 32;
         bool ok = true;
         for (int c = d.c0; c < d.c1; ++c, ++g) {
           const int b = g & 1;
@@ -595,8 +612,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ffn_kernel(const Params p) {
           tc_fence_after();
           const uint32_t a_tmem = tmem_base + kTmemA + b * kACols;
           const uint32_t b_addr = smem_u32(smem + kOffB + b * kBBytes);
-#pragma unroll
-          for (int s = 0; s < kChunkCols / 16; ++s)  // K = 16: 8 columns of A
+          const int ksteps = 2 * min(kChunkWords, W - kChunkWords * c);  // K = 16 each
+          for (int s = 0; s < ksteps; ++s)  // 8 columns of A per step
             mma_f16_ts(d_tmem, a_tmem + 8 * s, smem_desc(b_addr + s * 2 * d.np * 16, d.np * 16, 128),
                        idesc, (c > d.c0 || s > 0) ? 1u : 0u);
           mma_commit(&ab_empty[b]);
@@ -715,7 +732,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ffn_kernel(const Params p) {
       if (lane == 0) mbar_arrive(table_ready);
       if (!warp_wait(table_ready, vt & 1, abort_flag)) break;
 #define PW_DECODE(Q) \
-  decode_item<Q>(d.c0, d.c1, pl_full, pl_empty, a_full, ab_empty, abort_flag, g, tmem_base)
+  decode_item<Q>(d.c0, d.c1, p.m[d.mode].cols / 32, pl_full, pl_empty, a_full, ab_empty, \
+                 abort_flag, g, tmem_base)
       switch (d.q) {
         case 3: g = PW_DECODE(3); break;
         case 4: g = PW_DECODE(4); break;
