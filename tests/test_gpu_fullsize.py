@@ -38,15 +38,23 @@ def sampled_rows(L, idx, gate, tokens):
     return y
 
 
-@pytest.mark.parametrize("name,T,nsample", [("qwen15_moe_a2.7b", 32, 4),
-                                            ("qwen3_next_80b_a3b", 16, 4),
-                                            ("qwen2_57b_a14b", 64, 3),
-                                            ("mixtral_8x7b", 64, 3),
-                                            ("mixtral_8x7b", 256, 3)])
-def test_full_size_layer_sampled(torch_dev, name, T, nsample):
+# the last two are prefill-sized batches (the tensor-core FFN, several 64-token passes per
+# expert; routing by plain top-k, as a phase-aware schedule would do without the decode remap)
+@pytest.mark.parametrize("name,T,nsample,plain", [("qwen15_moe_a2.7b", 32, 4, False),
+                                                  ("qwen3_next_80b_a3b", 16, 4, False),
+                                                  ("qwen2_57b_a14b", 64, 3, False),
+                                                  ("mixtral_8x7b", 64, 3, False),
+                                                  ("mixtral_8x7b", 256, 3, False),
+                                                  ("mixtral_8x7b", 512, 2, True),
+                                                  ("qwen2_57b_a14b", 512, 2, True)])
+def test_full_size_layer_sampled(torch_dev, name, T, nsample, plain):
     torch, dev = torch_dev
+    import dataclasses
     from any_precision_expert_pw_b200.device_layer import DeviceLayer
+    from any_precision_expert_pw_b200.inputs import POLICY_NONE
     cfg = CONFIGS[name]
+    if plain:
+        cfg = dataclasses.replace(cfg, policy=POLICY_NONE, resident_frac=None)
     L = make_layer(cfg, T)
     D = DeviceLayer(L)
     D.forward()
