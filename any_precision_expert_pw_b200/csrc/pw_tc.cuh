@@ -56,9 +56,9 @@ constexpr int kPlaneWarp = 20;
 constexpr int kOperandWarp = 21;
 constexpr int kMmaWarp = 22;
 constexpr int kThreads = 23 * 32;
-// tensor memory: two accumulators of up to 64 fp32 columns, then two A buffers of 64 columns
-// (128 rows x 128 fp16)
-constexpr int kTmemCols = 512;  // 128 accumulator + 2 x 128 A columns used
+// tensor memory: two accumulators of up to 64 fp32 columns, then two A buffers of 128 columns
+// (128 rows x 256 fp16); the allocation is the next power of two, 512
+constexpr int kTmemCols = 512;
 constexpr int kTmemA = 2 * kPass;
 constexpr int kACols = kChunkCols / 2;
 constexpr int kPlaneStages = 3;
@@ -189,17 +189,8 @@ __device__ __forceinline__ uint32_t instr_desc(int n) {
   return (1u << 4) | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(kRows >> 4) << 24);
 }
 
-__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
-                                        uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-      ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// The same with A in tensor memory (a_tmem: lane 0, first column of the 128 x 16 slice).
+// D (tensor memory) = or += A (tensor memory; a_tmem: lane 0, first column of the 128 x 16
+// slice, two fp16 per column) x B (shared-memory descriptor) for one K = 16 step.
 __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
                                            uint32_t idesc, uint32_t accumulate) {
   asm volatile(
@@ -222,11 +213,6 @@ __device__ __forceinline__ void tc_fence_before() {
 }
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-// Generic-proxy writes to shared memory -> visible to the tensor core (async proxy).
-__device__ __forceinline__ void fence_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // 16 consecutive fp32 columns of this warp's tensor-memory lane quarter, one row per lane.

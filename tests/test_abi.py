@@ -97,3 +97,23 @@ def test_block_prepare_rejects_bad_blocks(libpw):
     assert B.pw_block_prepare(blk) == B.PW_OK                              # host-only check
     blk.planes = 4096 + 8
     assert B.pw_block_prepare(blk) == B.PW_ERR_INVALID_ARG                 # planes alignment
+
+
+def test_tc_switch_is_host_only(libpw):
+    # the FFN path switch is plain host state: no device call, negative values refused
+    assert B.pw_set_tc_min_tokens(0) == B.PW_OK
+    assert B.pw_set_tc_min_tokens(1 << 20) == B.PW_OK
+    assert B.pw_set_tc_min_tokens(-1) == B.PW_ERR_INVALID_ARG
+    assert B.pw_set_tc_min_tokens(4) == B.PW_OK          # the library default
+
+
+def test_workspace_holds_tensor_core_operands(libpw):
+    # the workspace has room for both FFN paths: among the rest, the fp16 operands of the
+    # tensor-core path, one row per padded position (each active expert's rows rounded up to 16)
+    for T, k, E, H, I in [(1, 2, 8, 4096, 14336), (64, 8, 64, 3584, 2560), (4, 2, 8, 256, 512),
+                          (512, 10, 512, 2048, 512)]:
+        ws = B.pw_moe_workspace_bytes(T, k, E, H, I)
+        tk = T * k
+        rows_pad = tk + 15 * min(E, tk)
+        assert ws >= 2 * rows_pad * (H + I) + 4 * tk * H * 8
+        assert ws % 256 == 0
