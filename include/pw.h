@@ -51,7 +51,7 @@ typedef struct CUstream_st* pw_stream_t; /* same object as cudaStream_t */
 typedef enum {
   PW_OK = 0,
   PW_ERR_INVALID_ARG = 1,  /* bad pointer, size, shape or config; nothing launched       */
-  PW_ERR_UNSUPPORTED = 2,  /* valid request outside what this build implements          */
+  PW_ERR_UNSUPPORTED = 2,  /* valid request outside what the library implements        */
   PW_ERR_CUDA = 3,         /* a CUDA runtime call failed (launch, sync, symbol copy)    */
   PW_ERR_NOT_RESIDENT = 4, /* device: a used block's page state is not PW_PAGE_GPU      */
   PW_ERR_TIMEOUT = 5,      /* device: a bounded wait gave up                            */
