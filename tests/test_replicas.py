@@ -76,3 +76,28 @@ def test_reference_arm_nonzero_rank_does_no_work(monkeypatch):
     with contextlib.redirect_stdout(out):
         assert bench.run_reference(args) is None
     assert out.getvalue() == ""
+
+
+def test_reference_arm_line_keeps_the_contract(monkeypatch):
+    # rank 0 of the reference arm (the oracle timed on the host) prints one JSON line with the
+    # keys the bench contract asks for; tiny layer, one step
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    monkeypatch.setenv("RANK", "0")
+    import json
+
+    import bench
+    args = types.SimpleNamespace(workload="tiny:4", steps=1, warmup=0, cpu_sample_rows=None,
+                                 affinity=False, no_rewrite=False)
+    out = io.StringIO()
+    with contextlib.redirect_stdout(out):
+        bench.run_reference(args)
+    lines = [ln for ln in out.getvalue().splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["value"] > 0
+    assert d["higher_is_better"] is True and d["n_gpus"] == 1 and d["steps"] == 1
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    assert d["e2e"]["value"] == d["value"]
+    assert "T=4" in d["config"]["workload"]
