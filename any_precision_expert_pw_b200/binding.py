@@ -40,7 +40,8 @@ EXPORTS = ("pw_block_prepare", "pw_pack_bitplanes", "pw_route_topk", "pw_topk", 
            "pw_plan_bitwidths",
            "pw_moe_workspace_bytes",
            "pw_moe_anyprec_forward",
-           "pw_moe_anyprec_forward_static", "pw_set_tc_min_tokens", "pw_commit_bits",
+           "pw_moe_anyprec_forward_static", "pw_set_tc_min_tokens", "pw_set_ffn_grid",
+           "pw_set_wait_limit_ns", "pw_test_hold_down_items", "pw_commit_bits",
            "pw_get_status",
            "pw_status_string", "pw_version")
 PW_STATIC_WORKSPACE_BYTES = 16 << 20
@@ -109,6 +110,9 @@ def lib() -> ctypes.CDLL:
         L.pw_moe_anyprec_forward.argtypes = [P, I, I, P, I, I, I, I, P, P, P, P, Z, S]
         L.pw_moe_anyprec_forward_static.argtypes = [P, I, I, P, I, I, I, I, P, P, P, S]
         L.pw_set_tc_min_tokens.argtypes = [I]
+        L.pw_set_ffn_grid.argtypes = [I]
+        L.pw_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+        L.pw_test_hold_down_items.argtypes = [I]
         L.pw_commit_bits.argtypes = [P, I, P, P, I, S]
         L.pw_page_copy.argtypes = [P, I, P, I, I, I, I, S]
         L.pw_page_update.argtypes = [P, I, P, I, S]
@@ -208,6 +212,21 @@ def pw_moe_anyprec_forward_static(pt_dev, layer, E, x_bf16, T, H, I, k, idx, gat
 
 def pw_set_tc_min_tokens(tokens_per_expert) -> int:
     return lib().pw_set_tc_min_tokens(tokens_per_expert)
+
+
+def pw_set_ffn_grid(ctas) -> int:
+    """Test hook: CTAs of the FFN launch (0 = one per SM)."""
+    return lib().pw_set_ffn_grid(ctas)
+
+
+def pw_set_wait_limit_ns(ns) -> int:
+    """Test hook: bound of the kernels' spin waits on the current device (0 = default 2 s)."""
+    return lib().pw_set_wait_limit_ns(int(ns))
+
+
+def pw_test_hold_down_items(extra) -> int:
+    """Test hook: down items wait for `extra` gate_up completions that never come (0 = off)."""
+    return lib().pw_test_hold_down_items(extra)
 
 
 def pw_commit_bits(pt_dev, num_blocks, block_ids, q, count, stream=0) -> int:

@@ -14,14 +14,36 @@
 
 namespace pw {
 
+// The tiled plane layout (pw.h, pw_block): 32-row tiles, stages of kTileStageWords words
+// (512 columns); inside a (tile, stage) run [plane][word][row], most significant plane first.
+constexpr int kTileRows = 32;
+constexpr int kTileStageWords = 16;
+constexpr int kTileStageCols = kTileStageWords * 32;
+
+// uint32 offset of (tile t, stage s, plane p, word u of the stage, row i) in a block of W
+// words per row holding n planes per run.
+__host__ __device__ __forceinline__ long long tiled_word(long long t, int s, int p, int u, int i,
+                                                         int n, int W) {
+  const int ws = (W - kTileStageWords * s) < kTileStageWords ? (W - kTileStageWords * s)
+                                                             : kTileStageWords;
+  return t * n * kTileRows * W + static_cast<long long>(s) * n * kTileRows * kTileStageWords +
+         static_cast<long long>(p) * kTileRows * ws + u * kTileRows + i;
+}
+
 // First device-side error wins; read and cleared by pw_get_status().
 __device__ int g_status = 0;
 
 __device__ __forceinline__ void set_status(int code) { atomicCAS(&g_status, 0, code); }
 
-// Bound on every spin wait: a wait that has not completed after this many nanoseconds of
-// global time records PW_ERR_TIMEOUT and gives up.  Normal waits finish in microseconds.
+// Bound on every spin wait: a wait that has not completed after g_wait_limit_ns nanoseconds of
+// global time records PW_ERR_TIMEOUT and gives up.  Normal waits finish in microseconds; the
+// default is 2 s, and pw_set_wait_limit_ns() (a test hook) shortens it.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+__device__ unsigned long long g_wait_limit_ns = kWaitLimitNs;
+
+// Test hook (pw_test_hold_down_items): extra gate_up completions a down item waits for, so that
+// its bounded wait runs out.  Zero in normal use.
+__device__ int g_test_hold = 0;
 
 __device__ __forceinline__ unsigned long long global_ns() {
   unsigned long long t;
@@ -68,16 +90,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+__device__ __forceinline__ unsigned long long wait_limit_ns() {
+  return *static_cast<volatile unsigned long long*>(&g_wait_limit_ns);
+}
+
 // Bounded wait for the phase of the given parity; false (and PW_ERR_TIMEOUT recorded) when
-// the limit ran out.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// the limit ran out.  With `abort_flag`, also gives up (false, nothing recorded) once another
+// thread of the CTA has set it.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          volatile int* abort_flag = nullptr) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
+  const unsigned long long limit = wait_limit_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 15u) == 0 && global_ns() - t0 > kWaitLimitNs) {
-      set_status(PW_ERR_TIMEOUT);
-      return false;
+    if ((it & 15u) == 0) {
+      if (abort_flag && *abort_flag) return false;
+      if (global_ns() - t0 > limit) {
+        set_status(PW_ERR_TIMEOUT);
+        return false;
+      }
     }
   }
 }

@@ -118,26 +118,36 @@ __device__ __forceinline__ void group_block(const pw_page_table* __restrict__ pt
 }
 
 // The one launch before the grouped FFN.  CTA 0 checks the page table and groups the
-// assignments; CTAs 1.. write X[t][xslot(c)] = x[t][c] as fp32 for c < H and 0 for
-// H <= c < ldx (one row per token: the gate_up producer maps a grouped position to its token),
-// and Hbuf[pos][c] = 0 for I <= c < ldh.  The FFN streams whole 1024-column stages, so the
-// padding must read as zero, and it reads activations in its decode order (xslot, a
-// permutation inside each 32-column group that keeps padding groups whole).  `vec`: x is
-// 16-byte aligned (H is a multiple of 128), so a thread converts 8 columns from one load.
-// The tensor-core FFN stages its activations with stage_x_kernel instead; it launches this
-// kernel with CTA 0 alone.
+// assignments; CTAs 1.. convert x to the CUDA-core FFN's activation layout: X[t] holds, per
+// 512-column stage, the stage's columns as fp16 (bf16 -> fp16 is exact for values in fp16's
+// normal range) in the decode's order (k4::xpos, a permutation inside each 32-column group),
+// with zeros for H <= c < ldx.  One row per token: the gate_up producer maps a grouped position
+// to its token.  `vec`: x is 16-byte aligned (H is a multiple of 128), so a thread converts 8
+// columns from one load.  The tensor-core FFN stages its activations with stage_x_kernel
+// instead; it launches this kernel with CTA 0 alone.
 __global__ void __launch_bounds__(kGroupThreads) setup_kernel(
     const pw_page_table* __restrict__ pt, int layer, const int32_t* __restrict__ idx, int T,
-    int k, int E, const uint16_t* __restrict__ x, int H, int ldx, int vec, float* __restrict__ X,
-    int I, int ldh, float* __restrict__ Hbuf, int32_t* __restrict__ counts,
-    int32_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ inv,
-    int32_t* __restrict__ active, int32_t* __restrict__ meta, int32_t* __restrict__ done,
-    PassOut po) {
+    int k, int E, const uint16_t* __restrict__ x, int H, int I, int ldx, int vec,
+    __half* __restrict__ X, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+    int32_t* __restrict__ perm, int32_t* __restrict__ inv, int32_t* __restrict__ active,
+    int32_t* __restrict__ meta, int32_t* __restrict__ done, PassOut po,
+    k4::ExpertDesc* __restrict__ xd) {
   griddep_wait();  // launched as a dependent of whatever precedes it in the stream
   griddep_launch();
   if (blockIdx.x == 0) {
     for (int e = threadIdx.x; e < E; e += blockDim.x) done[e] = 0;
     group_block(pt, layer, idx, T * k, k, E, po, counts, offsets, perm, inv, active, meta);
+    if (xd) {  // the CUDA-core FFN's per-(module, active expert) block descriptors
+      __syncthreads();
+      const int na = meta[0];
+      for (int i = threadIdx.x; i < 2 * na; i += blockDim.x) {
+        const int mode = i / na, a = i - mode * na;
+        const int e = active[a];
+        const int rows = mode == k4::MODE_GATE_UP ? 2 * I : H;
+        const int cols = mode == k4::MODE_GATE_UP ? H : I;
+        xd[mode * E + a] = k4::expert_desc(pt, layer, E, e, mode, rows, cols, counts[e], offsets[e]);
+      }
+    }
     return;
   }
   const size_t nthr = static_cast<size_t>(gridDim.x - 1) * blockDim.x;
@@ -145,7 +155,7 @@ __global__ void __launch_bounds__(kGroupThreads) setup_kernel(
   const int g8 = ldx / 8;  // 8-column groups per row
   for (size_t i = t0; i < static_cast<size_t>(T) * g8; i += nthr) {
     const size_t t = i / g8;
-    const int c = static_cast<int>(i - t * g8) * 8;  // columns c..c+7 share (c >> 3) & 3
+    const int c = static_cast<int>(i - t * g8) * 8;
     float v[8];
     if (c >= H) {
 #pragma unroll
@@ -162,19 +172,9 @@ __global__ void __launch_bounds__(kGroupThreads) setup_kernel(
 #pragma unroll
       for (int j = 0; j < 8; ++j) v[j] = bf16_to_f32(x[t * H + c + j]);
     }
-    // columns c+j and c+j+4 land in adjacent slots
-    float* row = X + t * ldx;
+    __half* row = X + t * ldx;
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
-      *reinterpret_cast<float2*>(row + k4::xslot(c + j)) = make_float2(v[j], v[j + 4]);
-  }
-  const int padh = ldh - I;
-  if (padh > 0) {
-    const size_t TK = static_cast<size_t>(T) * k;
-    for (size_t i = t0; i < TK * padh; i += nthr) {
-      const size_t pos = i / padh;
-      Hbuf[pos * ldh + I + (i - pos * padh)] = 0.0f;
-    }
+    for (int j = 0; j < 8; ++j) row[k4::xpos(c + j)] = __float2half_rn(v[j]);
   }
 }
 

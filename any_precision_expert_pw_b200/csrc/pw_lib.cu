@@ -80,6 +80,7 @@ pw_status device_info(DeviceInfo** out) {
 // Workspace layout of pw_moe_anyprec_forward.
 struct Workspace {
   size_t counts, offsets, perm, inv, active, meta, done, X, Hbuf, O;
+  size_t xd;                                         // CUDA-core path block descriptors
   size_t pbase, ptok, pnn, pass_tab, XB, HB, total;  // tensor-core path
   int ldx, ldh;
 };
@@ -87,6 +88,8 @@ struct Workspace {
 Workspace ws_layout(int T, int k, int E, int H, int I) {
   Workspace w;
   const size_t TK = static_cast<size_t>(T) * k;
+  // CUDA-core path activations (fp16, decode order): x per token, h per grouped position,
+  // rows padded to whole 512-column stages
   w.ldx = static_cast<int>(align_up(H, pw::k4::kStageCols));
   w.ldh = static_cast<int>(align_up(I, pw::k4::kStageCols));
   size_t o = 0;
@@ -102,9 +105,10 @@ Workspace ws_layout(int T, int k, int E, int H, int I) {
   w.active = take(4 * static_cast<size_t>(E));
   w.meta = take(32);  // [0] active experts, [1] valid assignments, [2] bad table, [4] work counter
   w.done = take(4 * static_cast<size_t>(E));  // gate_up tiles finished per active expert
-  w.X = take(4 * static_cast<size_t>(T) * w.ldx);
-  w.Hbuf = take(4 * TK * w.ldh);
+  w.X = take(2 * static_cast<size_t>(T) * w.ldx);
+  w.Hbuf = take(2 * TK * w.ldh);
   w.O = take(4 * TK * H * static_cast<size_t>(pw::k4::kMaxKSlices));
+  w.xd = take(sizeof(pw::k4::ExpertDesc) * 2 * static_cast<size_t>(E));
   // tensor-core path: each active expert's rows padded to a multiple of 16
   const size_t rows_pad = TK + 15 * std::min<size_t>(E, TK);
   w.pbase = take(4 * static_cast<size_t>(E));
@@ -127,9 +131,11 @@ std::mutex g_static_ws_mu;
 
 // Average routed tokens per active expert from which the tensor-core FFN is used.
 std::atomic<int> g_tc_min_tokens{4};
+// FFN launch grid override (test hook; 0 = one CTA per SM).
+std::atomic<int> g_ffn_grid{0};
 
 // k-slices for the down projection: fill the GPU in whole waves of work items, with at least
-// two 1024-column stages per slice.
+// two stages of the tiled layout (512 columns each) per slice.
 int choose_kslices(int items, int nst, int sms) {
   int best = 1;
   double best_eff = 0.0;
@@ -167,9 +173,10 @@ pw_status launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size
 pw_status launch_ffn(const pw::k4::Params& p, int max_active, int ntp, int sms,
                      cudaStream_t st) {
   long long items = 0;
-  for (int m = p.first_mode; m <= p.last_mode; ++m)
-    items += static_cast<long long>(max_active) * p.m[m].tiles * p.m[m].kslices;
-  const int grid = static_cast<int>(items < sms ? items : sms);
+  for (int m = pw::k4::MODE_GATE_UP; m <= pw::k4::MODE_DOWN; ++m)
+    items += static_cast<long long>(max_active) * p.m[m].pairs * p.m[m].kslices;
+  const int over = g_ffn_grid.load();
+  const int grid = over > 0 ? over : static_cast<int>(items < sms ? items : sms);
   if (ntp == 1)
     return launch_dependent(pw::k4::ffn_kernel<1>, dim3(grid), dim3(pw::k4::kThreads),
                             pw::k4::Layout<1>::kSmem, st, p);
@@ -178,6 +185,19 @@ pw_status launch_ffn(const pw::k4::Params& p, int max_active, int ntp, int sms,
                             pw::k4::Layout<2>::kSmem, st, p);
   return launch_dependent(pw::k4::ffn_kernel<4>, dim3(grid), dim3(pw::k4::kThreads),
                           pw::k4::Layout<4>::kSmem, st, p);
+}
+
+// Argument and shape checks shared by both forward entry points (the workspace is checked by
+// the caller): the same arguments give the same status from either.
+pw_status forward_args_status(const pw_page_table* pt_dev, int layer, int E,
+                              const uint16_t* x_bf16, int T, int H, int I, int k,
+                              const int32_t* idx, const float* gate, float* y) {
+  if (!pt_dev || !x_bf16 || !idx || !gate || !y) return PW_ERR_INVALID_ARG;
+  if (T < 1 || T > PW_MAX_TOKENS || k < 1 || k > PW_MAX_TOPK || layer < 0) return PW_ERR_INVALID_ARG;
+  if (E < 1 || E > PW_MAX_EXPERTS || k > E) return PW_ERR_INVALID_ARG;
+  if (H < 128 || I < 128 || H % 128 || I % 128) return PW_ERR_INVALID_ARG;
+  if (static_cast<long long>(T) * k > pw::kMaxAssign) return PW_ERR_UNSUPPORTED;
+  return PW_OK;
 }
 
 }  // namespace
@@ -230,11 +250,9 @@ pw_status pw_moe_anyprec_forward(const pw_page_table* pt_dev, int layer, int E,
                                  const uint16_t* x_bf16, int T, int H, int I, int k,
                                  const int32_t* idx, const float* gate, float* y, void* workspace,
                                  size_t ws_bytes, pw_stream_t stream) {
-  if (!pt_dev || !x_bf16 || !idx || !gate || !y || !workspace) return PW_ERR_INVALID_ARG;
-  if (T < 1 || T > PW_MAX_TOKENS || k < 1 || k > PW_MAX_TOPK || layer < 0) return PW_ERR_INVALID_ARG;
-  if (E < 1 || E > PW_MAX_EXPERTS || k > E) return PW_ERR_INVALID_ARG;
-  if (H < 128 || I < 128 || H % 128 || I % 128) return PW_ERR_INVALID_ARG;
-  if (static_cast<long long>(T) * k > pw::kMaxAssign) return PW_ERR_UNSUPPORTED;
+  const pw_status v = forward_args_status(pt_dev, layer, E, x_bf16, T, H, I, k, idx, gate, y);
+  if (v != PW_OK) return v;
+  if (!workspace) return PW_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(workspace) % 256) return PW_ERR_INVALID_ARG;
   const Workspace w = ws_layout(T, k, E, H, I);
   if (ws_bytes < w.total) return PW_ERR_INVALID_ARG;
@@ -249,8 +267,9 @@ pw_status pw_moe_anyprec_forward(const pw_page_table* pt_dev, int layer, int E,
   int32_t* active = reinterpret_cast<int32_t*>(base + w.active);
   int32_t* meta = reinterpret_cast<int32_t*>(base + w.meta);
   int32_t* done = reinterpret_cast<int32_t*>(base + w.done);
-  float* X = reinterpret_cast<float*>(base + w.X);
-  float* Hb = reinterpret_cast<float*>(base + w.Hbuf);
+  __half* X = reinterpret_cast<__half*>(base + w.X);
+  pw::k4::ExpertDesc* xd = reinterpret_cast<pw::k4::ExpertDesc*>(base + w.xd);
+  __half* Hb = reinterpret_cast<__half*>(base + w.Hbuf);
   float* O = reinterpret_cast<float*>(base + w.O);
   const int TK = T * k;
   const int max_active = E < TK ? E : TK;
@@ -266,14 +285,14 @@ pw_status pw_moe_anyprec_forward(const pw_page_table* pt_dev, int layer, int E,
 
   {
     // CTA 0 groups; the others convert x (8 columns per thread) for the CUDA-core FFN
-    const long long groups = static_cast<long long>(T) * (w.ldx / 8) +
-                             static_cast<long long>(TK) * (w.ldh - I) / 8;
+    const long long groups = static_cast<long long>(T) * (w.ldx / 8);
     const long long conv = (groups + pw::kGroupThreads - 1) / pw::kGroupThreads;
     const int grid =
         use_tc ? 1 : 1 + static_cast<int>(std::min<long long>(std::max(conv, 1LL), 2LL * di->sms));
     if (launch_dependent(pw::setup_kernel, dim3(grid), dim3(pw::kGroupThreads), 0, st, pt_dev,
-                         layer, idx, T, k, E, x_bf16, H, w.ldx, vec, X, I, w.ldh, Hb, counts,
-                         offsets, perm, inv, active, meta, done, po) != PW_OK)
+                         layer, idx, T, k, E, x_bf16, H, I, w.ldx, vec, X, counts,
+                         offsets, perm, inv, active, meta, done, po,
+                         use_tc ? static_cast<pw::k4::ExpertDesc*>(nullptr) : xd) != PW_OK)
       return PW_ERR_CUDA;
   }
   if (use_tc) {
@@ -324,7 +343,9 @@ pw_status pw_moe_anyprec_forward(const pw_page_table* pt_dev, int layer, int E,
     dn.out = O;
     dn.ld_out = H;
     dn.out_slice = static_cast<long long>(TK) * H;
-    if (launch_dependent(pw::k5::tc_ffn_kernel, dim3(di->sms), dim3(pw::k5::kThreads),
+    const int over = g_ffn_grid.load();
+    if (launch_dependent(pw::k5::tc_ffn_kernel, dim3(over > 0 ? over : di->sms),
+                         dim3(pw::k5::kThreads),
                          pw::k5::kSmem, st, q) != PW_OK)
       return PW_ERR_CUDA;
     const dim3 g((H + 255) / 256, T);
@@ -343,35 +364,42 @@ pw_status pw_moe_anyprec_forward(const pw_page_table* pt_dev, int layer, int E,
   p.meta = meta;
   p.sched = meta + 4;
   p.done = done;
+  p.one = 1;
+  p.xd = xd;
   // one launch: every gate_up item (h = SiLU(W_gate x) * (W_up x)), then every down item
   // (o = W_down h, split along k so that the work items fill the GPU); a down item streams h
-  // once all gate_up tiles of its expert are counted
-  p.first_mode = pw::k4::MODE_GATE_UP;
-  p.last_mode = pw::k4::MODE_DOWN;
+  // once all gate_up items of its expert are counted
   pw::k4::ModeParams& gu = p.m[pw::k4::MODE_GATE_UP];
   gu.rows = 2 * I;
   gu.cols = H;
   gu.half = I;
-  gu.tiles = I / pw::k4::kSegRows;
+  gu.pairs = I / 32;  // tile pairs: 32 gate rows and the 32 matching up rows
   gu.kslices = 1;
   gu.act = X;
   gu.ld_act = w.ldx;
   gu.act_map = perm;  // grouped position -> assignment t*k+slot -> token row of X
   gu.act_div = k;
-  gu.out = Hb;
-  gu.ld_out = w.ldh;
+  gu.hout = Hb;
+  gu.ld_hout = w.ldh;
+  gu.out = nullptr;
+  gu.ld_out = 0;
   gu.out_slice = 0;
   pw::k4::ModeParams& dn = p.m[pw::k4::MODE_DOWN];
   dn.rows = H;
   dn.cols = I;
   dn.half = 0;
-  dn.tiles = H / pw::k4::kRows;
-  dn.kslices = choose_kslices(max_active * dn.tiles,
-                              (I + pw::k4::kStageCols - 1) / pw::k4::kStageCols, di->sms);
+  dn.pairs = H / pw::k4::kItemRows;
+  // down items split along k to about the size of a gate_up item (64 rows x H columns): each
+  // item carries a fixed cost (its decode table, the first slot of its pipeline), so slicing
+  // finer than that costs more than the shorter end of the launch saves (measured)
+  dn.kslices = std::max(1, std::min({pw::k4::kMaxKSlices, (I + H / 2) / H,
+                                     (I + pw::k4::kStageCols - 1) / pw::k4::kStageCols / 2}));
   dn.act = Hb;
   dn.ld_act = w.ldh;
   dn.act_map = nullptr;
   dn.act_div = 1;
+  dn.hout = nullptr;
+  dn.ld_hout = 0;
   dn.out = O;
   dn.ld_out = H;
   dn.out_slice = static_cast<long long>(TK) * H;
@@ -390,7 +418,8 @@ pw_status pw_moe_anyprec_forward_static(const pw_page_table* pt_dev, int layer, 
                                         const uint16_t* x_bf16, int T, int H, int I, int k,
                                         const int32_t* idx, const float* gate, float* y,
                                         pw_stream_t stream) {
-  if (T < 1 || k < 1 || E < 1 || H < 1 || I < 1) return PW_ERR_INVALID_ARG;
+  const pw_status v = forward_args_status(pt_dev, layer, E, x_bf16, T, H, I, k, idx, gate, y);
+  if (v != PW_OK) return v;
   const size_t need = pw_moe_workspace_bytes(T, k, E, H, I);
   if (need == 0) return PW_ERR_INVALID_ARG;
   if (need > PW_STATIC_WORKSPACE_BYTES) return PW_ERR_UNSUPPORTED;  // shape too large for it
@@ -413,6 +442,24 @@ pw_status pw_set_tc_min_tokens(int tokens_per_expert) {
   if (tokens_per_expert < 0) return PW_ERR_INVALID_ARG;
   g_tc_min_tokens.store(tokens_per_expert);
   return PW_OK;
+}
+
+pw_status pw_set_ffn_grid(int ctas) {
+  if (ctas < 0) return PW_ERR_INVALID_ARG;
+  g_ffn_grid.store(ctas);
+  return PW_OK;
+}
+
+pw_status pw_set_wait_limit_ns(unsigned long long ns) {
+  const unsigned long long v = ns ? ns : pw::kWaitLimitNs;
+  return cudaMemcpyToSymbol(pw::g_wait_limit_ns, &v, sizeof(v)) == cudaSuccess ? PW_OK
+                                                                               : PW_ERR_CUDA;
+}
+
+pw_status pw_test_hold_down_items(int extra) {
+  if (extra < 0) return PW_ERR_INVALID_ARG;
+  return cudaMemcpyToSymbol(pw::g_test_hold, &extra, sizeof(extra)) == cudaSuccess ? PW_OK
+                                                                                   : PW_ERR_CUDA;
 }
 
 pw_status pw_commit_bits(pw_page_table* pt_dev, int num_blocks, const int32_t* block_ids,

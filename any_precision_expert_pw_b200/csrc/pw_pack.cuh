@@ -2,7 +2,7 @@
 // superposed bit-planes).  Plane p holds bit (n-1-p) of every index; column 32w+j of a row is
 // bit j of word w.  One warp builds the n words of a 32-column group with one ballot per plane
 // and stores them in the requested layout (PW_LAYOUT_ROWS, or the FFN's tiled layouts, where
-// the top planes of a 32-row tile and a 1024-column stage are one contiguous run).
+// the top planes of a 32-row tile and a 512-column stage are one contiguous run).
 #pragma once
 #include "pw_common.cuh"
 
@@ -22,11 +22,7 @@ __host__ __device__ __forceinline__ long long tiled_index(int layout, int rows, 
     t = r >> 5;
     i = r & 31;
   }
-  const int W = cols >> 5;
-  const int s = w >> 5, u = w & 31;
-  const int ws = (W - 32 * s) < 32 ? (W - 32 * s) : 32;
-  return static_cast<long long>(t) * n * 32 * W + static_cast<long long>(s) * n * 1024 +
-         static_cast<long long>(p) * 32 * ws + (u >> 1) * 64 + i * 2 + (u & 1);
+  return tiled_word(t, w / kTileStageWords, p, w % kTileStageWords, i, n, cols >> 5);
 }
 
 __global__ void __launch_bounds__(256) pack_bitplanes_kernel(const uint8_t* __restrict__ idx,

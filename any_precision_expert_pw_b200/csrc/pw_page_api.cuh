@@ -19,12 +19,13 @@ pw_status pw_page_copy(const uint32_t* src, int src_bits, uint32_t* dst, int dst
   const size_t W = static_cast<size_t>(cols) / 32, tiles = static_cast<size_t>(rows) / 32;
   const size_t src_tile = static_cast<size_t>(src_bits) * 32 * W * 4;
   const size_t dst_tile = static_cast<size_t>(dst_bits) * 32 * W * 4;
-  const size_t nst = (W + 31) / 32;
+  const size_t SW = pw::kTileStageWords;
+  const size_t nst = (W + SW - 1) / SW;
   for (size_t s = 0; s < nst; ++s) {
-    const size_t ws = std::min<size_t>(32, W - 32 * s);
+    const size_t ws = std::min<size_t>(SW, W - SW * s);
     const size_t width = static_cast<size_t>(q) * 32 * ws * 4;
-    const uint8_t* sp = reinterpret_cast<const uint8_t*>(src) + s * src_bits * 32 * 32 * 4;
-    uint8_t* dp = reinterpret_cast<uint8_t*>(dst) + s * dst_bits * 32 * 32 * 4;
+    const uint8_t* sp = reinterpret_cast<const uint8_t*>(src) + s * src_bits * 32 * SW * 4;
+    uint8_t* dp = reinterpret_cast<uint8_t*>(dst) + s * dst_bits * 32 * SW * 4;
     if (cudaMemcpy2DAsync(dp, dst_tile, sp, src_tile, width, tiles, cudaMemcpyDefault,
                           as_cuda(stream)) != cudaSuccess)
       return PW_ERR_CUDA;

@@ -21,7 +21,8 @@
 //   epilogue (4)           warp 16 + j reads rows 32j.. of the accumulator back (tensor-memory
 //                          lane quarter j): SiLU(gate) * up as fp16 into the down projection's
 //                          operand, or the down rows into the k-slice partials; warp 16 also
-//                          takes the items (first blockIdx.x, then a work counter), one ahead,
+//                          takes the items from a work counter (the first one included, so
+//                          only running CTAs own items), one ahead,
 //                          and prefetches the next item's LUT rows and first planes into L2;
 //   plane producer (1)     bulk-copies each chunk's top-q planes of the four tiles (4q runs of
 //                          1 KB in the tiled layout) into a ring of three stages;
@@ -232,7 +233,7 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   if (*abort_flag) return false;
-  if (!mbar_wait(bar, parity)) {
+  if (!mbar_wait(bar, parity, abort_flag)) {
     *abort_flag = 1;
     return false;
   }
@@ -259,12 +260,15 @@ template <int Q>
 __device__ __forceinline__ void decode_pair(uint32_t planes_off, uint32_t a_taddr, int t, int jj,
                                             int lane) {
   const int r = t * 32 + lane;  // row of the item's 128
-  // piece (t, p) = [word pair][row][2 words]: this warp's pair is 8 bytes per lane
-  const uint32_t off = planes_off + jj * 256 + lane * 8;
+  // piece (t, p) = [word][row]: words 2jj and 2jj + 1 of this lane's row, 4 bytes each (a
+  // warp's load is 128 contiguous bytes: conflict free)
+  const uint32_t off = planes_off + jj * 256 + lane * 4;
   uint2 P[Q];
 #pragma unroll
-  for (int p = 0; p < Q; ++p)
-    P[p] = *reinterpret_cast<const uint2*>(g_smem + off + (t * Q + p) * kPieceBytes);
+  for (int p = 0; p < Q; ++p) {
+    P[p].x = *reinterpret_cast<const uint32_t*>(g_smem + off + (t * Q + p) * kPieceBytes);
+    P[p].y = *reinterpret_cast<const uint32_t*>(g_smem + off + 128 + (t * Q + p) * kPieceBytes);
+  }
   // slot address of code v: 256v + 4 (r mod 64); the byte permute puts v in byte 1
   const uint32_t lbase = static_cast<uint32_t>((r & 63) * 4);
   const uint32_t psel = (t >> 1) ? 0x7632u : 0x5410u;  // high or low halves
@@ -370,7 +374,7 @@ __device__ __forceinline__ void build_part(const Desc& d, const ModeParams& mp, 
 }
 
 // L2 prefetch of what an item reads first: the LUT rows of its 128 rows and, for each of its
-// four tiles, the top q planes of its first 1024-column stage.
+// four tiles, the top q planes of its first 512-column stage.
 __device__ __forceinline__ void prefetch_item(const Params& p, const Desc& d) {
   if (!d.valid) return;
   const ModeParams& mp = p.m[d.mode];
@@ -381,10 +385,11 @@ __device__ __forceinline__ void prefetch_item(const Params& p, const Desc& d) {
   } else {
     prefetch_l2(d.lut + (static_cast<size_t>(d.mb * kRows) << d.q), kRows * row_bytes);
   }
-  const int W = mp.cols / 32, s = d.c0 * kChunkCols / 1024;
-  const int ws = min(32, W - 32 * s);
+  const int W = mp.cols / 32, s = d.c0 * kChunkCols / kTileStageCols;
+  const int ws = min(kTileStageWords, W - kTileStageWords * s);
   for (int t = 0; t < kTiles; ++t)
-    prefetch_l2(d.planes + t * d.tile_words + static_cast<size_t>(s) * d.n * 1024,
+    prefetch_l2(d.planes + t * d.tile_words +
+                    static_cast<size_t>(s) * d.n * kTileRows * kTileStageWords,
                 d.q * 32 * ws * 4);
 }
 
@@ -530,13 +535,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ffn_kernel(const Params p) {
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
-        const int s = c / 4;  // 1024-column stage of the tiled layout
-        const int ws = min(32, W - 32 * s);
+        constexpr int kChunksPerStage = kTileStageWords / kChunkWords;
+        const int s = c / kChunksPerStage;  // 512-column stage of the tiled layout
+        const int ws = min(kTileStageWords, W - kTileStageWords * s);
         if (lane < kTiles * d.q) {
           const int t = lane / d.q, pl = lane - t * d.q;
           const uint32_t* src = d.planes + t * d.tile_words +
-                                static_cast<size_t>(s) * d.n * 1024 + pl * 32 * ws +
-                                (c % 4) * kChunkWords * 32;
+                                static_cast<size_t>(s) * d.n * kTileRows * kTileStageWords +
+                                pl * kTileRows * ws + (c % kChunksPerStage) * kChunkWords * 32;
           bulk_g2s(smem + kOffPlanes + ps * kPlaneStageBytes + (t * d.q + pl) * kPieceBytes, src,
                    min(kChunkWords, W - kChunkWords * c) * 128, &pl_full[ps]);
         }
@@ -620,9 +626,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ffn_kernel(const Params p) {
     Desc next;  // warp 16, lane 0: the item claimed for the next descriptor
     if (ew == 0 && lane == 0) {
       next.item = -1;
-      if (static_cast<int>(blockIdx.x) < n_items) {
-        next = resolve(p, blockIdx.x, npass);
-        next.item = blockIdx.x;
+      const int it0 = atomicAdd(p.sched, 1);  // every item comes from the counter
+      if (it0 < n_items) {
+        next = resolve(p, it0, npass);
+        next.item = it0;
         prefetch_item(p, next);
       }
     }
@@ -639,7 +646,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ffn_kernel(const Params p) {
           slot = next;
           mbar_arrive(&desc_full[j % kDescRing]);
           if (next.item >= 0) {
-            const int it2 = gridDim.x + atomicAdd(p.sched, 1);
+            const int it2 = atomicAdd(p.sched, 1);
             next.item = -1;
             if (it2 < n_items) {
               next = resolve(p, it2, npass);

@@ -96,15 +96,16 @@ enum { PW_ACT_HIT = 0, PW_ACT_FETCH = 1, PW_ACT_SUBST = 2 };
  *   significant), so the top q planes give the q-bit index = top q bits of the parent index.
  *   In PW_LAYOUT_ROWS a plane is uint32 [rows][cols/32] and column 32w+j sits at bit j of
  *   word w.  The FFN reads the same words rearranged so that everything one CTA needs for a
- *   32-row tile and a 1024-column stage is one contiguous run, most significant plane first:
+ *   32-row tile and a 512-column stage is one contiguous run, most significant plane first:
  *     tile t, row i of the tile:  PW_LAYOUT_TILED_DOWN    -> block row 32t + i;
  *                                 PW_LAYOUT_TILED_GATE_UP -> gate row 16t + i for i < 16,
  *                                                            up row I + 16t + (i - 16) otherwise;
- *     stage s = words 32s .. 32s + ws - 1 of each row, ws = min(32, cols/32 - 32s);
- *     word w = 32s + 2j + h of plane p, row i of tile t sits at uint32 index
- *       t * (n * 32 * cols/32) + s * (n * 32 * 32) + p * (32 * ws) + j * 64 + i * 2 + h
+ *     stage s = words 16s .. 16s + ws - 1 of each row, ws = min(16, cols/32 - 16s);
+ *     word w = 16s + u of plane p, row i of tile t sits at uint32 index
+ *       t * (n * 32 * cols/32) + s * (n * 32 * 16) + p * (32 * ws) + u * 32 + i
  *     (n = parent_bits).  Reading the top q planes of (t, s) reads the first q * 32 * ws words
- *     of that run.  `layout` holds PW_LAYOUT_TILED_GATE_UP or PW_LAYOUT_TILED_DOWN; the
+ *     of that run; inside it a plane is [word][row], so one word of 32 consecutive rows is 128
+ *     contiguous bytes.  `layout` holds PW_LAYOUT_TILED_GATE_UP or PW_LAYOUT_TILED_DOWN; the
  *     forward checks it against the module.  `planes` is 16-byte aligned.
  *   stored_bits: how many planes each (tile, stage) run holds in `planes` (0 = parent_bits):
  *     a block paged in at bitwidth q (pw_page_copy) keeps only its top q planes on the device,
@@ -336,6 +337,30 @@ pw_status pw_moe_anyprec_forward_static(const pw_page_table* pt_dev, int layer, 
 pw_status pw_set_tc_min_tokens(int tokens_per_expert);
 
 /* ---------------------------------------------------------------------------------------
+ * Test hooks (no counterpart on the pages).  They exist so that the tests can reach paths that
+ * a healthy run never takes; production code leaves them at their defaults.
+ *
+ * pw_set_ffn_grid: number of CTAs of the FFN launch of pw_moe_anyprec_forward (both paths);
+ *   0 (default) = one per SM (capped by the work items on the CUDA-core path).  A grid larger
+ *   than the GPU can hold at once (more than one CTA per SM never fits) checks that the
+ *   gate_up -> down dependency does not assume every CTA to be resident.  Process-wide, host
+ *   state only; takes effect on later calls.  Negative -> PW_ERR_INVALID_ARG.
+ *
+ * pw_set_wait_limit_ns: bound of every spin wait in libpw's kernels on the current device
+ *   (a wait that has not completed within it records PW_ERR_TIMEOUT and gives up, and the
+ *   work it guarded writes zeros).  0 restores the default of 2 s.  Synchronous (a copy to a
+ *   device variable); call it between launches, not during stream capture.
+ *
+ * pw_test_hold_down_items: every down item of the fused FFN launch on the current device waits
+ *   for `extra` more gate_up completions than exist, so its bounded wait runs out and the
+ *   forward ends with PW_ERR_TIMEOUT (the failure path of a gate_up tile that never finishes).
+ *   0 (default) restores normal behaviour.  Synchronous, like pw_set_wait_limit_ns.
+ * ------------------------------------------------------------------------------------- */
+pw_status pw_set_ffn_grid(int ctas);
+pw_status pw_set_wait_limit_ns(unsigned long long ns);
+pw_status pw_test_hold_down_items(int extra);
+
+/* ---------------------------------------------------------------------------------------
  * pw_commit_bits [PW1][PW3]: set committed_bits of `count` blocks (device arrays block_ids
  * [count] int32 and q [count] uint8), stream-ordered, so that a commit takes effect exactly
  * between two forward calls on the stream (a safe boundary).  A block id out of range or a q
@@ -361,7 +386,7 @@ typedef struct pw_page_update_t {
  * every (tile, stage) run between two buffers of the same block in the tiled layout holding
  * src_bits and dst_bits planes per run (q <= both): host -> device (page in at bitwidth q,
  * the device copy keeping only q planes per run), device -> host, device -> device.  Host
- * buffers must be pinned for the copy to be asynchronous.  One pitched copy per 1024-column
+ * buffers must be pinned for the copy to be asynchronous.  One pitched copy per 512-column
  * stage, on `stream`.  rows % 32 == 0, cols % 128 == 0, both pointers 16-byte aligned.
  * ------------------------------------------------------------------------------------- */
 pw_status pw_page_copy(const uint32_t* src, int src_bits, uint32_t* dst, int dst_bits, int rows,

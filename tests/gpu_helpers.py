@@ -7,7 +7,7 @@ from any_precision_expert_pw_b200.inputs import CONFIGS
 FFN_RTOL_RMS = 2e-3        # max |y_gpu - y_ref| <= 2e-3 * rms(y_ref)
 GATE_ATOL = 1e-6           # routing gates (fp32 vs float64, rounded once on both sides)
 
-# scaled-down shapes: several tiles, ragged column tails (H or I not a multiple of 1024)
+# scaled-down shapes: several tiles, ragged column tails (H or I not a multiple of 512)
 SCALED = {
     "tiny": CONFIGS["tiny"],
     "qwen15": CONFIGS["qwen15_moe_a2.7b"].scaled(H=640, I=384),
@@ -33,8 +33,8 @@ def assert_ffn_close(y_gpu, y_ref, what=""):
 
 def tiled_reference(planes, layout):
     """The tiled arrangement of [n][rows][words] bit-planes, built with array reshapes: row
-    tiles of 32 (gate_up: 16 gate rows then the 16 matching up rows), stages of 32 words, and
-    inside a stage [plane][word pair][row][2]."""
+    tiles of 32 (gate_up: 16 gate rows then the 16 matching up rows), stages of 16 words, and
+    inside a stage [plane][word][row]."""
     n, R, W = planes.shape
     if layout == B.PW_LAYOUT_TILED_GATE_UP:
         half = R // 2
@@ -45,8 +45,7 @@ def tiled_reference(planes, layout):
     tiles = planes[:, order, :].reshape(n, R // 32, 32, W)
     out = []
     for t in range(R // 32):
-        for s0 in range(0, W, 32):
-            blk = tiles[:, t, :, s0:s0 + 32]                      # [n][32][ws]
-            ws = blk.shape[2]
-            out.append(blk.reshape(n, 32, ws // 2, 2).transpose(0, 2, 1, 3).reshape(-1))
+        for s0 in range(0, W, 16):
+            blk = tiles[:, t, :, s0:s0 + 16]                      # [n][32 rows][ws words]
+            out.append(blk.transpose(0, 2, 1).reshape(-1))        # [n][ws][32]
     return np.concatenate(out)
