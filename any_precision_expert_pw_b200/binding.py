@@ -99,12 +99,12 @@ def lib() -> ctypes.CDLL:
         L.pw_route_topk.argtypes = [P, P, P, I, I, I, ctypes.POINTER(pw_route_cfg), P, P, P, S]
         L.pw_topk.argtypes = [P, I, I, ctypes.POINTER(pw_route_cfg), P, P, S]
         L.pw_substitute.argtypes = [P, P, P, P, I, I, ctypes.POINTER(pw_route_cfg), P, P, S]
-        L.pw_remap.argtypes = [P, P, P, I, I, ctypes.POINTER(pw_route_cfg), P, S]
+        L.pw_remap.argtypes = [P, P, P, I, I, ctypes.POINTER(pw_route_cfg), P, P, S]
         L.pw_affinity_default.argtypes = [I, I, ctypes.POINTER(pw_affinity_cfg)]
         L.pw_cache_step.argtypes = [P, P, P, I, I, ctypes.POINTER(pw_route_cfg), ctypes.c_double,
                                     P, P, P, I, P, P, P, S]
         L.pw_affinity_remap.argtypes = [P, P, P, I, I, ctypes.POINTER(pw_route_cfg),
-                                        ctypes.POINTER(pw_affinity_cfg), P, P, S]
+                                        ctypes.POINTER(pw_affinity_cfg), P, P, P, S]
         L.pw_moe_workspace_bytes.argtypes = [I, I, I, I, I]
         L.pw_moe_workspace_bytes.restype = Z
         L.pw_moe_anyprec_forward.argtypes = [P, I, I, P, I, I, I, I, P, P, P, P, Z, S]
@@ -173,17 +173,19 @@ def pw_substitute(logits, idx, gate, resident, T, E, cfg, action, mass, stream=0
     return lib().pw_substitute(logits, idx, gate, resident, T, E, _cfg(cfg), action, mass, stream)
 
 
-def pw_remap(logits, idx, gate, T, E, cfg, critical, stream=0) -> int:
-    return lib().pw_remap(logits, idx, gate, T, E, _cfg(cfg), critical, stream)
+def pw_remap(logits, idx, gate, T, E, cfg, critical, unique=0, stream=0) -> int:
+    """unique: device int32[2] receiving the distinct experts before / after (0 = none)."""
+    return lib().pw_remap(logits, idx, gate, T, E, _cfg(cfg), critical, unique, stream)
 
 
 def pw_affinity_default(E, k, out) -> int:
     return lib().pw_affinity_default(E, k, _cfg(out))
 
 
-def pw_affinity_remap(logits, idx, gate, T, E, cfg, acfg, critical, bins, stream=0) -> int:
+def pw_affinity_remap(logits, idx, gate, T, E, cfg, acfg, critical, bins, unique=0,
+                      stream=0) -> int:
     return lib().pw_affinity_remap(logits, idx, gate, T, E, _cfg(cfg), _cfg(acfg), critical,
-                                   bins, stream)
+                                   bins, unique, stream)
 
 
 def pw_cache_step(logits, idx, gate, T, E, cfg, beta, resident, mass, freq, capacity, action,

@@ -24,9 +24,11 @@
 //   decode (16 warps)   warp w takes word w (32 columns) of every stage, both rows of its lane;
 //   reducer (1 warp)    adds the sixteen per-warp partial sums of every pass in a fixed order
 //                       and writes the output (SiLU(gate) * up for gate_up).
-// Activations are fp16 (gate_up: x, bf16 -> fp16, exact in fp16's normal range; down: h
-// rounded once from fp32, relative error <= 2^-11) and every product is one fma.rn.f32.f16:
-// the fp16 weight times the fp16 activation, exact, added in fp32.
+// Activations are fp16 (gate_up: x, bf16 -> fp16, exact in fp16's normal range; down: h as a
+// pair hi + lo of fp16 values, hi = fp16(h), lo = fp16(h - hi), so the products keep h to about
+// 22 bits -- a single fp16 rounding of h leaves the whole output of some batches at the edge of
+// the parity bar) and every product is one fma.rn.f32.f16: the fp16 weight times the fp16
+// activation, exact, added in fp32.
 // Decode tables hold fp16 LUT values; slot s of lane i sits at byte 256 s + 128 u + 4 i (u =
 // table buffer), so a gather of 32 lanes is conflict free and its address is one byte
 // permute of the code byte.  After an 8x8 bit transpose of plane words, byte k of register j
@@ -52,10 +54,10 @@ constexpr int kProducerWarp = kDecodeWarps + kLutWarps;
 constexpr int kReducerWarp = kProducerWarp + 1;
 constexpr int kThreads = (kReducerWarp + 1) * 32;
 constexpr int kTableBytes = 256 * 256;                     // 256 slots x 256-byte stride
-constexpr int kXBytes = kStageCols * 2;                    // fp16 activations, one stage/token
+constexpr int kXBytes = kStageCols * 2;                    // fp16 x, one stage, one token
+constexpr int kXBytesDown = 2 * kXBytes;                   // h: 512 hi then 512 lo
 constexpr int kSlotPlaneBytes = kTiles * PW_MAX_BITS * kStageWords * 128;  // 32 KB
-constexpr int kMaxSubStages = 2;  // stages per slot (q <= 4)
-constexpr int kMaxKSlices = 16;
+constexpr int kMaxKSlices = 8;
 constexpr int kDescRing = 8;    // item descriptors in flight (LUT warps -> every other role)
 
 // The kernel's dynamic shared memory, named directly (not through a pointer) wherever the
@@ -92,13 +94,14 @@ struct Desc {
 };
 static_assert(sizeof(Desc) == 88, "descriptor size");
 
-// Stages per slot for a block of committed bitwidth q.
-__host__ __device__ __forceinline__ int sub_stages(int q) { return q <= 4 ? 2 : 1; }
+// Stages per slot for a block of committed bitwidth q, at most ms (the layout's).
+__host__ __device__ __forceinline__ int sub_stages(int q, int ms) { return q <= 4 ? ms : 1; }
 
 template <int NTP>
 struct Layout {
-  static constexpr int kStages = NTP == 4 ? 3 : 4;  // slots
-  static constexpr int kSlotBytes = kSlotPlaneBytes + NTP * kMaxSubStages * kXBytes;
+  static constexpr int kStages = NTP == 1 ? 4 : 3;  // slots
+  static constexpr int kMaxSub = NTP == 4 ? 1 : 2;   // stages per slot at most (q <= 4)
+  static constexpr int kSlotBytes = kSlotPlaneBytes + NTP * kMaxSub * kXBytesDown;
   static constexpr int kRedBytes = 2 * kDecodeWarps * NTP * kTiles * 32 * 4;
   static constexpr int kDescBytes = kDescRing * static_cast<int>(sizeof(Desc));
   static constexpr int kBarBytes = (2 * kStages + 8 + 2 * kDescRing) * 8 + 32;
@@ -343,8 +346,8 @@ __device__ __forceinline__ void fma4(uint32_t w0, uint32_t w1, uint32_t wb0, uin
 
 // One word (32 columns) of rows a and b of this lane, NT tokens.  pa / pb: byte offsets of the
 // word's most significant plane in the two tiles (planes pstride apart); xs: the word's fp16
-// activations of token 0 (xstride bytes between tokens).
-template <int Q, int NT>
+// activations of token 0 (xstride bytes between tokens; DOWN: the lo parts 1024 bytes on).
+template <int Q, int NT, bool DOWN>
 __device__ __forceinline__ void decode_word(uint32_t pa, uint32_t pb, uint32_t pstride,
                                             uint32_t xs, uint32_t xstride, uint32_t lane_base,
                                             uint32_t m1, uint32_t m2, uint32_t m4,
@@ -388,6 +391,14 @@ __device__ __forceinline__ void decode_word(uint32_t pa, uint32_t pb, uint32_t p
           fma4<PAIR, 1>(w0, w1, wb0, wb1, x0, x1, acc[t]);
         else
           fma4<PAIR, 0>(w0, w1, wb0, wb1, x0, x1, acc[t]);
+        if constexpr (DOWN) {
+          const uint4 xl = lds_u128(xs + 1024 + t * xstride + i * 16);
+          const uint32_t y0 = (k >> 1) ? xl.y : xl.x, y1 = (k >> 1) ? xl.w : xl.z;
+          if (k & 1)
+            fma4<PAIR, 1>(w0, w1, wb0, wb1, y0, y1, acc[t]);
+          else
+            fma4<PAIR, 0>(w0, w1, wb0, wb1, y0, y1, acc[t]);
+        }
       }
     }
   }
@@ -395,7 +406,8 @@ __device__ __forceinline__ void decode_word(uint32_t pa, uint32_t pb, uint32_t p
 
 // Byte offsets inside a slot holding stages s, s + 1 (m of them) of an item at bitwidth q: tile
 // 2P's planes of sub-stage j at j q 2 KB, tile 2P + 1's m q 2 KB further on, then the
-// activation chunk of token t and sub-stage j at 2 m q 2 KB + (t m + j) KB.
+// activation chunk of token t and sub-stage j at 2 m q 2 KB + (t m + j) xunit (xunit: 1 KB of
+// x for gate_up, 2 KB of h hi and lo for down).
 __host__ __device__ __forceinline__ uint32_t slot_tile_b(int q, int m) {
   return static_cast<uint32_t>(m * q * kStageWords * 128);
 }
@@ -406,13 +418,14 @@ __host__ __device__ __forceinline__ uint32_t slot_x(int q, int m) { return 2 * s
 // ring slot g % NS and holds M = sub_stages(Q) consecutive stages.  At the end it waits until
 // the reducer has freed the partial-sum buffer (rfree, phase rphase) and writes the warp's sums
 // of rows a and b per token there; the caller advances its slot counter by the item's units.
-template <int Q, int NT, int NS>
+template <int Q, int NT, int NS, int MS, bool DOWN>
 __device__ __noinline__ void run_stages(uint64_t* full, uint64_t* empty,
                                         volatile int* abort_flag, uint32_t slot_bytes,
                                         int words_total, uint32_t lane_base, int s0, int s1,
                                         uint32_t g, uint32_t one, float* part, uint64_t* rfree,
                                         uint32_t rphase) {
-  constexpr int M = Q <= 4 ? 2 : 1;
+  constexpr int M = Q <= 4 ? MS : 1;
+  constexpr int XU = DOWN ? kXBytesDown : kXBytes;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t m1 = one << 1, m2 = one << 2, m4 = one << 4;
   float acc[NT][4];
@@ -428,9 +441,9 @@ __device__ __noinline__ void run_stages(uint64_t* full, uint64_t* empty,
       const int ws = min(kStageWords, words_total - (s + j) * kStageWords);
       if (warp < ws) {
         const uint32_t pa = st + j * Q * kStageWords * 128 + warp * 128 + lane * 4;
-        decode_word<Q, NT>(pa, pa + M * Q * kStageWords * 128, ws * 128,
-                           st + 2 * M * Q * kStageWords * 128 + j * kXBytes + warp * 64,
-                           M * kXBytes, lane_base, m1, m2, m4, acc);
+        decode_word<Q, NT, DOWN>(pa, pa + M * Q * kStageWords * 128, ws * 128,
+                                 st + 2 * M * Q * kStageWords * 128 + j * XU + warp * 64,
+                                 M * XU, lane_base, m1, m2, m4, acc);
       }
     }
     __syncwarp();
@@ -448,20 +461,34 @@ __device__ __noinline__ void run_stages(uint64_t* full, uint64_t* empty,
   full, empty, abort_flag, LY::kSlotBytes, words_total, lane_base, d.s0, d.s1, g, one, part,  \
       rfree, rphase
 
+template <int NT, int NTP, bool DOWN>
+__device__ __forceinline__ void run_qm(const Desc& d, uint64_t* full, uint64_t* empty,
+                                       volatile int* abort_flag, int words_total,
+                                       uint32_t lane_base, uint32_t g, uint32_t one, float* part,
+                                       uint64_t* rfree, uint32_t rphase) {
+  using LY = Layout<NTP>;
+  constexpr int NS = LY::kStages, MS = LY::kMaxSub;
+  switch (d.q) {
+    case 3: run_stages<3, NT, NS, MS, DOWN>(PW_RUN_ARGS); break;
+    case 4: run_stages<4, NT, NS, MS, DOWN>(PW_RUN_ARGS); break;
+    case 5: run_stages<5, NT, NS, MS, DOWN>(PW_RUN_ARGS); break;
+    case 6: run_stages<6, NT, NS, MS, DOWN>(PW_RUN_ARGS); break;
+    case 7: run_stages<7, NT, NS, MS, DOWN>(PW_RUN_ARGS); break;
+    default: run_stages<8, NT, NS, MS, DOWN>(PW_RUN_ARGS); break;
+  }
+}
+
 template <int NT, int NTP>
 __device__ __forceinline__ void run_q(const Desc& d, uint64_t* full, uint64_t* empty,
                                       volatile int* abort_flag, int words_total,
                                       uint32_t lane_base, uint32_t g, uint32_t one, float* part,
                                       uint64_t* rfree, uint32_t rphase) {
-  using LY = Layout<NTP>;
-  switch (d.q) {
-    case 3: run_stages<3, NT, LY::kStages>(PW_RUN_ARGS); break;
-    case 4: run_stages<4, NT, LY::kStages>(PW_RUN_ARGS); break;
-    case 5: run_stages<5, NT, LY::kStages>(PW_RUN_ARGS); break;
-    case 6: run_stages<6, NT, LY::kStages>(PW_RUN_ARGS); break;
-    case 7: run_stages<7, NT, LY::kStages>(PW_RUN_ARGS); break;
-    default: run_stages<8, NT, LY::kStages>(PW_RUN_ARGS); break;
-  }
+  if (d.mode == MODE_DOWN)
+    run_qm<NT, NTP, true>(d, full, empty, abort_flag, words_total, lane_base, g, one, part,
+                          rfree, rphase);
+  else
+    run_qm<NT, NTP, false>(d, full, empty, abort_flag, words_total, lane_base, g, one, part,
+                           rfree, rphase);
 }
 #undef PW_RUN_ARGS
 
@@ -552,9 +579,13 @@ __device__ __forceinline__ void store_table(const LutRegs& r, int q, uint32_t u,
   }
 }
 
-// h of feature f, rounded once to fp16, at its place in the down projection's activations.
+// h of feature f at its place in the down projection's activations: per 512-column stage,
+// 512 hi values then 512 lo values (hi = fp16(h), lo = fp16(h - hi)), xpos order inside.
 __device__ __forceinline__ void store_h(__half* hrow, int f, float h) {
-  hrow[xpos(f)] = __float2half_rn(h);
+  const __half hi = __float2half_rn(h);
+  __half* c = hrow + (f / kStageCols) * (2 * kStageCols) + xpos(f % kStageCols);
+  c[0] = hi;
+  c[kStageCols] = __float2half_rn(h - __half2float(hi));
 }
 
 template <int NTP>
@@ -664,14 +695,15 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
           arow_mode = cur.te <= NTP ? cur.mode : -1;
           arow_a = cur.a;
         }
-        const int m = sub_stages(cur.q);
+        const int m = sub_stages(cur.q, LY::kMaxSub);
         const uint32_t tb = slot_tile_b(cur.q, m), xo = slot_x(cur.q, m);
+        const uint32_t xu = cur.mode == MODE_DOWN ? kXBytesDown : kXBytes;
         for (int s = cur.s0; s < cur.s1; s += m, ++g) {
           const int slot = g % LY::kStages;
           wait_bar(&empty[slot], ((g / LY::kStages) & 1) ^ 1, abort_flag);
           uint8_t* st = ring + slot * LY::kSlotBytes;
           const int nsub = min(m, cur.s1 - s);
-          uint32_t bytes = ntok * nsub * kXBytes;
+          uint32_t bytes = ntok * nsub * xu;
           for (int j = 0; j < nsub; ++j)
             bytes += 2 * cur.q * min(kStageWords, words_total - (s + j) * kStageWords) * 128;
           mbar_arrive_expect_tx(&full[slot], bytes);
@@ -683,8 +715,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
             bulk_g2s(st + sub, pa + soff, pbytes, &full[slot]);
             bulk_g2s(st + tb + sub, pb + soff, pbytes, &full[slot]);
             for (int t = 0; t < ntok; ++t)
-              bulk_g2s(st + xo + (t * m + j) * kXBytes,
-                       arow[t] + static_cast<size_t>(s + j) * kXBytes, kXBytes, &full[slot]);
+              bulk_g2s(st + xo + (t * m + j) * xu, arow[t] + static_cast<size_t>(s + j) * xu, xu,
+                       &full[slot]);
           }
         }
         if (*abort_flag) break;
@@ -843,7 +875,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
         run_q<(NTP >= 4 ? 4 : 1), NTP>(d, full, empty, abort_flag, words_total, lane_base, g,
                                        one, part, rfree, rphase);
       {
-        const int m = sub_stages(d.q);
+        const int m = sub_stages(d.q, LY::kMaxSub);
         g += (d.s1 - d.s0 + m - 1) / m;
       }
       if (ch + NTP >= d.te) {  // last pass over this item: release the table

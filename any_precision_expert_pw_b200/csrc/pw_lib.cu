@@ -88,10 +88,10 @@ struct Workspace {
 Workspace ws_layout(int T, int k, int E, int H, int I) {
   Workspace w;
   const size_t TK = static_cast<size_t>(T) * k;
-  // CUDA-core path activations (fp16, decode order): x per token, h per grouped position,
-  // rows padded to whole 512-column stages
+  // CUDA-core path activations (fp16, decode order): x per token, h (hi and lo parts) per
+  // grouped position, rows padded to whole 512-column stages
   w.ldx = static_cast<int>(align_up(H, pw::k4::kStageCols));
-  w.ldh = static_cast<int>(align_up(I, pw::k4::kStageCols));
+  w.ldh = static_cast<int>(2 * align_up(I, pw::k4::kStageCols));
   size_t o = 0;
   auto take = [&](size_t bytes) {
     const size_t at = o;
@@ -116,7 +116,7 @@ Workspace ws_layout(int T, int k, int E, int H, int I) {
   w.pnn = take(4 * rows_pad);
   w.pass_tab = take(4 * (std::min<size_t>(E, TK) + TK / pw::kPassTokens + 1));
   w.XB = take(2 * rows_pad * H);
-  w.HB = take(2 * rows_pad * I);
+  w.HB = take(2 * 2 * rows_pad * I);  // h as hi and lo fp16 parts
   w.total = o;
   return w;
 }

@@ -321,18 +321,38 @@ __global__ void __launch_bounds__(256) substitute_kernel(
 
 constexpr int kRemapMaxAssign = 8192;  // T * k of the single-CTA batch rewrites
 
+// Number of distinct experts among the TK assignments (idx_s: shared copy, or idx: global,
+// read after the CTA's own writes); `flags` [E] and `n` are shared scratch.  CTA-wide: every
+// thread calls it, and every thread gets the count.
+__device__ __forceinline__ int distinct_experts(const int16_t* idx_s, const int32_t* idx, int TK,
+                                                int E, uint8_t* flags, int* n) {
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) flags[e] = 0;
+  if (threadIdx.x == 0) *n = 0;
+  __syncthreads();
+  for (int a = threadIdx.x; a < TK; a += blockDim.x) flags[idx_s ? idx_s[a] : idx[a]] = 1;
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    if (flags[e]) atomicAdd(n, 1);
+  __syncthreads();
+  return *n;
+}
+
 // Single CTA: batch gate sums, critical set, then one warp per token remaps (E <= 32 * PL).
 template <int PL>
 __global__ void __launch_bounds__(1024) remap_kernel(const float* __restrict__ logits,
                                                      int32_t* __restrict__ idx,
                                                      const float* __restrict__ gate, int T, int E,
                                                      int k, int critical_n,
-                                                     uint8_t* __restrict__ critical) {
+                                                     uint8_t* __restrict__ critical,
+                                                     int32_t* __restrict__ unique) {
   __shared__ double S[PW_MAX_EXPERTS];
   __shared__ uint8_t r0[PW_MAX_EXPERTS];
   __shared__ uint8_t crit[PW_MAX_EXPERTS];
+  __shared__ uint8_t used[PW_MAX_EXPERTS];
   __shared__ int16_t idx_s[kRemapMaxAssign];  // the assignments, scanned once per expert
   __shared__ int n_r0;
+  __shared__ int n_used;
   __shared__ int bad;
   const int tid = threadIdx.x;
   const int TK = T * k;
@@ -352,6 +372,7 @@ __global__ void __launch_bounds__(1024) remap_kernel(const float* __restrict__ l
     if (tid == 0) set_status(PW_ERR_BAD_EXPERT);
     return;
   }
+  const int before = unique ? distinct_experts(idx_s, nullptr, TK, E, used, &n_used) : 0;
   for (int t = tid; t < T; t += blockDim.x) r0[idx_s[t * k]] = 1;
   // S_e: float64, ascending (token, slot) order -- one thread per expert scans the batch.
   for (int e = tid; e < E; e += blockDim.x) {
@@ -404,6 +425,13 @@ __global__ void __launch_bounds__(1024) remap_kernel(const float* __restrict__ l
     if (lane == 0)
       for (int s = 1; s < k; ++s) idx[static_cast<size_t>(t) * k + s] = cur[s];
   }
+  if (unique) {
+    const int after = distinct_experts(nullptr, idx, TK, E, used, &n_used);
+    if (tid == 0) {
+      unique[0] = before;
+      unique[1] = after;
+    }
+  }
 }
 
 // LYNX AffinityBinning (2.1, 2.2): per-token confidence bins from the top-2 logit gap, batch
@@ -414,13 +442,16 @@ template <int PL>
 __global__ void __launch_bounds__(1024) affinity_remap_kernel(
     const float* __restrict__ logits, int32_t* __restrict__ idx, const float* __restrict__ gate,
     int T, int E, int k, int critical_n, int B, double w, int low,
-    uint8_t* __restrict__ critical, int32_t* __restrict__ bins_out) {
+    uint8_t* __restrict__ critical, int32_t* __restrict__ bins_out,
+    int32_t* __restrict__ unique) {
   __shared__ double S[PW_MAX_EXPERTS];
   __shared__ uint8_t r0[PW_MAX_EXPERTS];
   __shared__ uint8_t crit[PW_MAX_EXPERTS];
+  __shared__ uint8_t used[PW_MAX_EXPERTS];
   __shared__ uint8_t bin_s[PW_MAX_TOKENS];
   __shared__ int16_t idx_s[kRemapMaxAssign];
   __shared__ int n_r0;
+  __shared__ int n_used;
   __shared__ int bad;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
   const int TK = T * k;
@@ -440,6 +471,7 @@ __global__ void __launch_bounds__(1024) affinity_remap_kernel(
     if (tid == 0) set_status(PW_ERR_BAD_EXPERT);
     return;
   }
+  const int before = unique ? distinct_experts(idx_s, nullptr, TK, E, used, &n_used) : 0;
   // confidence bins: warp per token, gap between the two largest logits (fp32)
   for (int t = warp; t < T; t += nw) {
     WarpRow<PL> row;
@@ -533,6 +565,13 @@ __global__ void __launch_bounds__(1024) affinity_remap_kernel(
     __syncwarp();
     if (lane == 0)
       for (int s = 1; s < k; ++s) idx[static_cast<size_t>(t) * k + s] = cur[s];
+  }
+  if (unique) {
+    const int after = distinct_experts(nullptr, idx, TK, E, used, &n_used);
+    if (tid == 0) {
+      unique[0] = before;
+      unique[1] = after;
+    }
   }
 }
 

@@ -66,7 +66,8 @@ pw_status pw_substitute(const float* logits, int32_t* idx, const float* gate,
 }
 
 pw_status pw_remap(const float* logits, int32_t* idx, const float* gate, int T, int E,
-                   const pw_route_cfg* cfg, uint8_t* critical, pw_stream_t stream) {
+                   const pw_route_cfg* cfg, uint8_t* critical, int32_t* unique,
+                   pw_stream_t stream) {
   if (!logits || !idx || !gate) return PW_ERR_INVALID_ARG;
   if (T < 1 || T > PW_MAX_TOKENS || E < 1 || E > PW_MAX_EXPERTS || !cfg_ok(cfg, E))
     return PW_ERR_INVALID_ARG;
@@ -74,7 +75,7 @@ pw_status pw_remap(const float* logits, int32_t* idx, const float* gate, int T, 
   cudaStream_t st = as_cuda(stream);
 #define PW_REMAP(PL)                                                                          \
   pw::remap_kernel<PL><<<1, 1024, 0, st>>>(logits, idx, gate, T, E, cfg->k, cfg->critical_n, \
-                                           critical)
+                                           critical, unique)
   if (E <= 32) PW_REMAP(1);
   else if (E <= 64) PW_REMAP(2);
   else if (E <= 128) PW_REMAP(4);
@@ -122,7 +123,8 @@ pw_status pw_affinity_default(int E, int k, pw_affinity_cfg* out) {
 
 pw_status pw_affinity_remap(const float* logits, int32_t* idx, const float* gate, int T, int E,
                             const pw_route_cfg* cfg, const pw_affinity_cfg* acfg,
-                            uint8_t* critical, int32_t* bins, pw_stream_t stream) {
+                            uint8_t* critical, int32_t* bins, int32_t* unique,
+                            pw_stream_t stream) {
   if (!logits || !idx || !gate || !acfg) return PW_ERR_INVALID_ARG;
   if (T < 1 || T > PW_MAX_TOKENS || E < 1 || E > PW_MAX_EXPERTS || !cfg_ok(cfg, E))
     return PW_ERR_INVALID_ARG;
@@ -134,7 +136,7 @@ pw_status pw_affinity_remap(const float* logits, int32_t* idx, const float* gate
 #define PW_AFF(PL)                                                                            \
   pw::affinity_remap_kernel<PL><<<1, 1024, 0, st>>>(logits, idx, gate, T, E, cfg->k,          \
                                                     cfg->critical_n, acfg->num_bins, w,        \
-                                                    acfg->low_bins, critical, bins)
+                                                    acfg->low_bins, critical, bins, unique)
   if (E <= 32) PW_AFF(1);
   else if (E <= 64) PW_AFF(2);
   else if (E <= 128) PW_AFF(4);

@@ -26,12 +26,20 @@
 //                          and prefetches the next item's LUT rows and first planes into L2;
 //   plane producer (1)     bulk-copies each chunk's top-q planes of the four tiles (4q runs of
 //                          1 KB in the tiled layout) into a ring of three stages;
-//   operand producer (1)   bulk-copies each chunk's activations (np * 512 contiguous bytes);
+//   operand producer (1)   bulk-copies each chunk's activations (np * 512 contiguous bytes;
+//                          for down, h as hi + lo fp16 parts, one block per 32-token sub-pass);
 //                          a down item first waits until every gate_up item of its expert is
 //                          counted;
-//   MMA (1)                one thread issues 16 tcgen05.mma (K = 16 each) per chunk into one of
-//                          two accumulators and commits each chunk's completion to the barrier
-//                          that frees its A and B buffers.
+//   MMA (1)                one thread issues 16 tcgen05.mma (K = 16 each) per chunk and operand
+//                          part into one of two accumulators and commits each operand block's
+//                          completion to the barrier that frees its B buffer, each chunk's to the
+//                          one that frees its A buffer.
+// The down projection's activations h are fp32 results of the gate_up epilogue; they are held as
+// hi = fp16(h) and lo = fp16(h - hi) and multiplied as two operands into the same accumulator,
+// so the products keep h to about 22 bits (a single fp16 rounding of h, 2^-11 relative, leaves
+// the whole output of a large batch at the edge of the parity bar).  A pass of more than 32
+// tokens is split into two sub-passes of 32 + the rest (MMA N of 32 and np - 32), each of
+// whose hi and lo blocks of a chunk fit one B buffer.
 // The decode table pairs rows r and r + 64 of the item: the 32-bit slot at byte 256v + 4r
 // (r < 64) holds (LUT_r[v], LUT_{r+64}[v]).  A warp's 32 rows are 32 consecutive r mod 64, so
 // its gathers hit 32 different banks, the slot address is one byte permute of the code byte,
@@ -84,7 +92,7 @@ struct ModeParams {
   int mblocks;   // 128-row blocks per expert
   int kslices;   // k-slices per block (1 for gate_up)
   const __half* bsrc;  // operand staging [padded rows][cols], chunk order (stage_x_kernel)
-  __half* hout;        // gate_up: the down projection's operand staging [padded rows][I]
+  __half* hout;        // gate_up: the down projection's operand staging, 2 I per padded row
   float* out;          // down: [kslice][pos][ld_out]
   int ld_out;
   long long out_slice;
@@ -116,9 +124,10 @@ struct Desc {
 static_assert(sizeof(Desc) == 96, "descriptor size");
 
 constexpr int kOffBar = kOffDesc + kDescRing * static_cast<int>(sizeof(Desc));
-// barriers: pl_full[4] pl_empty[4] b_full[2] ab_empty[2] a_full[2] acc_full[2] acc_empty[2]
-// table_ready table_free desc_full[8] desc_free[8] mma_done; then the TMEM address and abort
-constexpr int kNumBars = 2 * kPlaneStages + 10 + 2 + 2 * kDescRing + 1;
+// barriers: pl_full[3] pl_empty[3] b_full[2] ab_empty[2] a_full[2] acc_full[2] acc_empty[2]
+// b_empty[2] table_ready table_free desc_full[8] desc_free[8] mma_done; then the TMEM address
+// and the abort flag
+constexpr int kNumBars = 2 * kPlaneStages + 12 + 2 + 2 * kDescRing + 1;
 constexpr int kSmem = kOffBar + kNumBars * 8 + 16;
 static_assert(kSmem <= 227 * 1024, "shared memory budget");
 static_assert(kOffB % 1024 == 0 && kOffPlanes % 1024 == 0, "alignment");
@@ -156,7 +165,8 @@ __device__ __forceinline__ Desc resolve(const Params& p, int item, int npass) {
   const int nch = (mp.cols + kChunkCols - 1) / kChunkCols;  // a last chunk may hold 128 columns
   d.c0 = (nch * d.ks) / mp.kslices;
   d.c1 = (nch * (d.ks + 1)) / mp.kslices;
-  d.bsrc = mp.bsrc + static_cast<size_t>(d.prow0) * mp.cols;
+  // gate_up operand: cols fp16 per padded row; down: hi and lo, 2 cols per padded row
+  d.bsrc = mp.bsrc + static_cast<size_t>(d.prow0) * mp.cols * (mode == MODE_DOWN ? 2 : 1);
   const pw_block* b = p.pt->blocks + (static_cast<size_t>(p.layer) * p.E + e) * 2 + mode;
   d.q = b->committed_bits;
   d.n = b->stored_bits ? b->stored_bits : b->parent_bits;
@@ -393,6 +403,23 @@ __device__ __forceinline__ void prefetch_item(const Params& p, const Desc& d) {
                 d.q * 32 * ws * 4);
 }
 
+// Place of h element (token n of the pass, feature f) in the down operand staging, relative to
+// the pass's first padded row (2 I fp16 per padded row): sub-pass sp = n / 32 of a pass of
+// more than 32 tokens (sub-pass 0 then holds 32 rows), then per 256-column chunk one block of
+// np_s rows hi followed by np_s rows lo, each in the MMA's K-major core-matrix order.
+struct HPlace {
+  size_t hi, lo;
+};
+__device__ __forceinline__ HPlace h_place(int np, int I, int n, int f) {
+  const int sp = (np > 32 && n >= 32) ? 1 : 0;
+  const int nps = np > 32 ? (sp ? np - 32 : 32) : np;
+  const int nn = n - 32 * sp;
+  const int c = f / kChunkCols, cc = min(kChunkCols, I - c * kChunkCols);
+  const size_t blk = static_cast<size_t>(sp) * 64 * I + static_cast<size_t>(c) * 2 * nps * kChunkCols;
+  const size_t in = static_cast<size_t>((f % kChunkCols) / 8) * nps * 8 + nn * 8 + (f % 8);
+  return {blk + in, blk + static_cast<size_t>(nps) * cc + in};
+}
+
 // Epilogue of one item, warp j (rows 32j.. of the accumulator).  gate_up: lanes 0-15 hold the
 // gate rows and lanes 16-31 the matching up rows of features 16 * tile + lane; h = SiLU(gate)
 // * up goes to the down operand staging as fp16, padding tokens included (they are zeros).
@@ -407,15 +434,17 @@ __device__ __forceinline__ void epilogue(const Desc& d, const ModeParams& mp, in
     if (d.mode == MODE_GATE_UP) {
       const int f = tile * 16 + (lane & 15);
       // the down operand has I = mp.half columns
-      __half* base = mp.hout + static_cast<size_t>(d.prow0) * mp.half +
-                     (f / kChunkCols) * d.np * kChunkCols + ((f % kChunkCols) / 8) * d.np * 8 +
-                     (f % 8);
+      __half* base = mp.hout + static_cast<size_t>(d.prow0) * 2 * mp.half;
 #pragma unroll
       for (int n = 0; n < 16; ++n) {
         const float up = __shfl_down_sync(0xffffffffu, v[n], 16);
         if (lane < 16) {
           const float g = v[n];
-          base[(c0 + n) * 8] = __float2half_rn(g / (1.0f + expf(-g)) * up);
+          const float h = g / (1.0f + expf(-g)) * up;
+          const __half hi = __float2half_rn(h);
+          const HPlace pl = h_place(d.np, mp.half, c0 + n, f);
+          base[pl.hi] = hi;
+          base[pl.lo] = __float2half_rn(h - __half2float(hi));
         }
       }
     } else {
@@ -435,9 +464,12 @@ __device__ __forceinline__ void zero_outputs(const Desc& d, const ModeParams& mp
   if (d.mode == MODE_GATE_UP) {
     if (lane >= 16) return;
     const int f = tile * 16 + lane;
-    __half* base = mp.hout + static_cast<size_t>(d.prow0) * mp.half +
-                   (f / kChunkCols) * d.np * kChunkCols + ((f % kChunkCols) / 8) * d.np * 8 + (f % 8);
-    for (int n = 0; n < d.np; ++n) base[n * 8] = __float2half_rn(0.0f);
+    __half* base = mp.hout + static_cast<size_t>(d.prow0) * 2 * mp.half;
+    for (int n = 0; n < d.np; ++n) {
+      const HPlace pl = h_place(d.np, mp.half, n, f);
+      base[pl.hi] = __float2half_rn(0.0f);
+      base[pl.lo] = __float2half_rn(0.0f);
+    }
   } else {
     float* base = mp.out + d.ks * mp.out_slice + static_cast<size_t>(d.pos0) * mp.ld_out +
                   tile * 32 + lane;
@@ -456,7 +488,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ffn_kernel(const Params p) {
   uint64_t* a_full = ab_empty + 2;
   uint64_t* acc_full = a_full + 2;
   uint64_t* acc_empty = acc_full + 2;
-  uint64_t* table_ready = acc_empty + 2;
+  uint64_t* b_empty = acc_empty + 2;  // [2] B buffer read by its MMAs (MMA -> operand producer)
+  uint64_t* table_ready = b_empty + 2;
   uint64_t* table_free = table_ready + 1;
   uint64_t* desc_full = table_free + 1;
   uint64_t* desc_free = desc_full + kDescRing;
@@ -477,6 +510,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ffn_kernel(const Params p) {
     for (int b = 0; b < 2; ++b) {
       mbar_init(&b_full[b], 1);
       mbar_init(&ab_empty[b], 1);
+      mbar_init(&b_empty[b], 1);
       mbar_init(&a_full[b], kDecodeWarps);
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], kEpiWarps);
@@ -565,16 +599,24 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ffn_kernel(const Params p) {
         if (!d.valid) continue;
         // the down operand (h) of this expert is complete once all its gate_up items count
         if (d.mode == MODE_DOWN && !k4::wait_count(p.done + d.a, d.target, abort_flag)) break;
-        const int W = p.m[d.mode].cols / 32;
+        const int W = p.m[d.mode].cols / 32, I2 = 2 * p.m[d.mode].cols;
+        const bool down = d.mode == MODE_DOWN;
+        const int nsp = down && d.np > 32 ? 2 : 1;
         bool ok = true;
-        for (int c = d.c0; c < d.c1; ++c, ++g) {
-          const int b = g & 1;
-          // np rows x the chunk's columns (256, or 128 for a last half chunk) of fp16
-          const uint32_t bytes = d.np * min(kChunkWords, W - kChunkWords * c) * 64;
-          if (!(ok = wait_bar(&ab_empty[b], ((g >> 1) & 1) ^ 1, abort_flag))) break;
-          mbar_arrive_expect_tx(&b_full[b], bytes);
-          bulk_g2s(smem + kOffB + b * kBBytes,
-                   d.bsrc + static_cast<size_t>(c) * d.np * kChunkCols, bytes, &b_full[b]);
+        for (int c = d.c0; ok && c < d.c1; ++c) {
+          const int cc = min(kChunkWords, W - kChunkWords * c) * 32;  // the chunk's columns
+          for (int sp = 0; sp < nsp; ++sp, ++g) {
+            const int b = g & 1;
+            const int nps = nsp == 2 ? (sp ? d.np - 32 : 32) : d.np;
+            // gate_up: np rows x cc columns of fp16 x; down: the hi and lo blocks of a sub-pass
+            const uint32_t bytes = (down ? 2 : 1) * nps * cc * 2;
+            const __half* src =
+                down ? d.bsrc + static_cast<size_t>(sp) * 32 * I2 + static_cast<size_t>(c) * 2 * nps * kChunkCols
+                     : d.bsrc + static_cast<size_t>(c) * d.np * kChunkCols;
+            if (!(ok = wait_bar(&b_empty[b], ((g >> 1) & 1) ^ 1, abort_flag))) break;
+            mbar_arrive_expect_tx(&b_full[b], bytes);
+            bulk_g2s(smem + kOffB + b * kBBytes, src, bytes, &b_full[b]);
+          }
         }
         if (!ok) break;
       }
@@ -583,7 +625,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ffn_kernel(const Params p) {
   } else if (warp == kMmaWarp) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      uint32_t g = 0, va = 0;
+      uint32_t g = 0, va = 0, ga = 0;  // B blocks, valid items, chunks (A buffers)
       for (uint32_t j = 0;; ++j) {
         if (!wait_bar(&desc_full[j % kDescRing], (j / kDescRing) & 1, abort_flag)) break;
         const Desc d = cdesc[j % kDescRing];
@@ -593,22 +635,44 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ffn_kernel(const Params p) {
         const uint32_t acc = va & 1;
         if (!wait_bar(&acc_empty[acc], ((va >> 1) & 1) ^ 1, abort_flag)) break;
         tc_fence_after();
-        const uint32_t idesc = instr_desc(d.np);
         const uint32_t d_tmem = tmem_base + acc * kPass;
         const int W = p.m[d.mode].cols / 32;
+        const bool down = d.mode == MODE_DOWN;
+        const int nsp = down && d.np > 32 ? 2 : 1;
         bool ok = true;
-        for (int c = d.c0; c < d.c1; ++c, ++g) {
-          const int b = g & 1;
-          if (!(ok = wait_bar(&a_full[b], (g >> 1) & 1, abort_flag))) break;
-          if (!(ok = wait_bar(&b_full[b], (g >> 1) & 1, abort_flag))) break;
-          tc_fence_after();
-          const uint32_t a_tmem = tmem_base + kTmemA + b * kACols;
-          const uint32_t b_addr = smem_u32(smem + kOffB + b * kBBytes);
+        for (int c = d.c0; ok && c < d.c1; ++c, ++ga) {
+          const int ab = ga & 1;
+          if (!(ok = wait_bar(&a_full[ab], (ga >> 1) & 1, abort_flag))) break;
+          const uint32_t a_tmem = tmem_base + kTmemA + ab * kACols;
           const int ksteps = 2 * min(kChunkWords, W - kChunkWords * c);  // K = 16 each
-          for (int s = 0; s < ksteps; ++s)  // 8 columns of A per step
-            mma_f16_ts(d_tmem, a_tmem + 8 * s, smem_desc(b_addr + s * 2 * d.np * 16, d.np * 16, 128),
-                       idesc, (c > d.c0 || s > 0) ? 1u : 0u);
-          mma_commit(&ab_empty[b]);
+          const int cc = ksteps * 16;
+          for (int sp = 0; sp < nsp; ++sp, ++g) {
+            const int b = g & 1;
+            if (!(ok = wait_bar(&b_full[b], (g >> 1) & 1, abort_flag))) break;
+            tc_fence_after();
+            const uint32_t b_addr = smem_u32(smem + kOffB + b * kBBytes);
+            if (!down) {
+              const uint32_t idesc = instr_desc(d.np);
+              for (int s = 0; s < ksteps; ++s)  // 8 columns of A per step
+                mma_f16_ts(d_tmem, a_tmem + 8 * s,
+                           smem_desc(b_addr + s * 2 * d.np * 16, d.np * 16, 128), idesc,
+                           (c > d.c0 || s > 0) ? 1u : 0u);
+            } else {
+              // sub-pass sp: tokens 32 sp .. of the pass, accumulator columns 32 sp ..; its hi
+              // block then its lo block, into the same accumulator
+              const int nps = nsp == 2 ? (sp ? d.np - 32 : 32) : d.np;
+              const uint32_t idesc = instr_desc(nps);
+              for (int part = 0; part < 2; ++part) {
+                const uint32_t pb = b_addr + part * nps * cc * 2;
+                for (int s = 0; s < ksteps; ++s)
+                  mma_f16_ts(d_tmem + 32 * sp, a_tmem + 8 * s,
+                             smem_desc(pb + s * 2 * nps * 16, nps * 16, 128), idesc,
+                             (c > d.c0 || part > 0 || s > 0) ? 1u : 0u);
+              }
+            }
+            mma_commit(&b_empty[b]);
+          }
+          if (ok) mma_commit(&ab_empty[ab]);  // the chunk's A buffer is read
         }
         if (!ok) break;
         mma_commit(&acc_full[acc]);

@@ -91,6 +91,8 @@ class DeviceLayer:
         self.action = torch.empty((T, k), dtype=u8, device=self.device)
         self.mass = torch.empty((T,), dtype=f32, device=self.device)
         self.critical = torch.empty((E,), dtype=u8, device=self.device)
+        self.unique = torch.zeros((2,), dtype=i32, device=self.device)  # distinct experts
+                                                                        # before / after a remap
         self.y = torch.empty((T, H), dtype=f32, device=self.device)
         self.ws_bytes = B.pw_moe_workspace_bytes(T, k, E, H, self.I)
         self.workspace = torch.empty((self.ws_bytes,), dtype=u8, device=self.device)
@@ -112,12 +114,13 @@ class DeviceLayer:
             B.check(B.pw_affinity_default(self.E, self.k, acfg), "pw_affinity_default")
             B.check(B.pw_affinity_remap(self.logits.data_ptr(), self.idx.data_ptr(),
                                         self.gate.data_ptr(), self.T, self.E, self.route_cfg,
-                                        acfg, self.critical.data_ptr(), 0, self.stream),
+                                        acfg, self.critical.data_ptr(), 0,
+                                        self.unique.data_ptr(), self.stream),
                     "pw_affinity_remap")
         elif pol == POLICY_REMAP:
             B.check(B.pw_remap(self.logits.data_ptr(), self.idx.data_ptr(), self.gate.data_ptr(),
                                self.T, self.E, self.route_cfg, self.critical.data_ptr(),
-                               self.stream), "pw_remap")
+                               self.unique.data_ptr(), self.stream), "pw_remap")
         elif pol != POLICY_NONE:
             B.check(B.pw_substitute(self.logits.data_ptr(), self.idx.data_ptr(),
                                     self.gate.data_ptr(), self.resident.data_ptr(), self.T,

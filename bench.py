@@ -119,7 +119,10 @@ def recorded_traffic(workload_key: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+    """nvidia-smi clocks / throttle reasons sampled every 100 ms around the timed region.  The
+    timed region of a short run can be shorter than one sampling interval, so the caller keeps
+    the GPU on the same step (untimed) until samples() has grown by `min_samples` since the
+    timed region began; only those samples are reported."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -129,8 +132,9 @@ class ClockSampler:
         self.gpu_id = gpu_id
         self.proc = None
         self.path = None
+        self.skip = 0
 
-    def start(self):
+    def start(self, first_sample_timeout_s: float = 5.0):
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
@@ -140,10 +144,30 @@ class ClockSampler:
                  "-lms", "100", "-i", self.gpu_id], stdout=self.fh, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+            return
+        t0 = time.time()   # nvidia-smi takes a moment to print its first line
+        while self.samples() == 0 and time.time() - t0 < first_sample_timeout_s:
+            if self.proc.poll() is not None:
+                break
+            time.sleep(0.05)
+
+    def samples(self) -> int:
+        if self.proc is None or self.path is None:
+            return 0
+        try:
+            self.fh.flush()
+            with open(self.path) as f:
+                return sum(1 for line in f if line.count(",") >= 8)
+        except Exception:
+            return 0
+
+    def mark(self):
+        """Only samples written after this call are reported."""
+        self.skip = self.samples()
 
     def stop(self):
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -152,10 +176,9 @@ class ClockSampler:
         self.fh.close()
         sms, mx, reasons = [], None, set()
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for line in open(self.path):
+        lines = [line for line in open(self.path) if line.count(",") >= 8][self.skip:]
+        for line in lines:
             f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
             try:
                 sms.append(float(f[1]))
                 mx = float(f[2])
@@ -306,7 +329,8 @@ def run_pw(args):
     from any_precision_expert_pw_b200 import binding as B
     from any_precision_expert_pw_b200.accounting import ffn_bytes, layer_bytes, plane_bytes
     from any_precision_expert_pw_b200.device_layer import DeviceLayer
-    from any_precision_expert_pw_b200.inputs import POLICY_NONE, make_layer
+    from any_precision_expert_pw_b200.inputs import (POLICY_AFFINITY, POLICY_NONE, POLICY_REMAP,
+                                                     make_layer)
 
     rep = Replicas("nccl")
     world, rank, local = rep.world, rep.rank, rep.local
@@ -375,15 +399,26 @@ def run_pw(args):
     uuid = str(getattr(torch.cuda.get_device_properties(dev), "uuid", local))
     gpu_id = uuid if uuid.startswith("GPU-") else (f"GPU-{uuid}" if len(uuid) > 30 else str(local))
     clocks = ClockSampler(gpu_id)
+    clocks.start()
     barrier()
     torch.cuda.synchronize(dev)
-    clocks.start()
+    clocks.mark()
     t_wall0 = time.perf_counter()
     evs = timed(g_step, args.steps)
     torch.cuda.synchronize(dev)
     barrier()
     t_wall1 = time.perf_counter()
+    # a short timed region sees no sample: keep the GPU on the same step (untimed) until three
+    # samples cover the region and what follows it, at most 3 s
+    t_keep = time.perf_counter()
+    extra_steps = 0
+    while clocks.samples() - clocks.skip < 3 and time.perf_counter() - t_keep < 3.0:
+        timed(g_step, 20)
+        torch.cuda.synchronize(dev)
+        extra_steps += 20
     clk = clocks.stop()
+    clk["window"] = ("timed region" if extra_steps == 0 else
+                     f"timed region + {extra_steps} untimed replays of the same step")
     step_ms = max_over_ranks(mean_ms(evs))
     step_med_ms = max_over_ranks(median_ms(evs))
 
@@ -433,6 +468,8 @@ def run_pw(args):
         "config": {"workload": f"{cfg.name}-shaped MoE decode layer, T={T}", "H": cfg.H,
                    "E": cfg.E, "I": cfg.I, "k": cfg.k, "parent_bits": cfg.n,
                    "bits": L.q.tolist(), "experts_used": used.tolist(),
+                   **({"distinct_experts_before_after_rewrite": D.unique.cpu().tolist()}
+                      if cfg.policy in (POLICY_REMAP, POLICY_AFFINITY) else {}),
                    "ffn_path": "tensor-core (tcgen05)" if tc_path else "cuda-core",
                    "rewrite": {-1: "none", 0: "fetch-all", 1: "0.15 rule", 2: "first choice",
                                3: "batch remap", 4: "AffinityBinning remap"}[cfg.policy],

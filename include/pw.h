@@ -211,10 +211,13 @@ pw_status pw_substitute(const float* logits, int32_t* idx, const float* gate,
  * index), keeping its gate; with none left the slot is kept.  Every token keeps exactly k
  * distinct experts.
  *   logits [T][E] fp32, idx [T][k] int32 (in/out), gate [T][k] fp32, critical [E] uint8
- *   (may be NULL).  Runs as one thread block: T * k <= 8192.
+ *   (may be NULL), unique int32[2] (may be NULL): the number of distinct experts the batch
+ *   routes to before and after the remap -- the experts whose weights the FFN reads.
+ *   Runs as one thread block: T * k <= 8192.
  * ------------------------------------------------------------------------------------- */
 pw_status pw_remap(const float* logits, int32_t* idx, const float* gate, int T, int E,
-                   const pw_route_cfg* cfg, uint8_t* critical, pw_stream_t stream);
+                   const pw_route_cfg* cfg, uint8_t* critical, int32_t* unique,
+                   pw_stream_t stream);
 
 /* AffinityBinning configuration (pw_affinity_remap). */
 typedef struct pw_affinity_cfg {
@@ -240,12 +243,14 @@ pw_status pw_affinity_default(int E, int k, pw_affinity_cfg* out);
  *         ascending (token, slot) order;
  *   critical set C and the remap as in pw_remap with S_e in place of the gate sums, applied
  *   only to tokens with bin_t < low_bins.  With w = +inf this is exactly pw_remap.
- *   logits [T][E] fp32, idx [T][k] int32 (in/out), gate [T][k] fp32, critical [E] uint8 and
- *   bins [T] int32 outputs (either may be NULL).  One thread block: T * k <= 8192.
+ *   logits [T][E] fp32, idx [T][k] int32 (in/out), gate [T][k] fp32, critical [E] uint8,
+ *   bins [T] int32 and unique int32[2] (distinct experts before / after, as in pw_remap)
+ *   outputs (each may be NULL).  One thread block: T * k <= 8192.
  * ------------------------------------------------------------------------------------- */
 pw_status pw_affinity_remap(const float* logits, int32_t* idx, const float* gate, int T, int E,
                             const pw_route_cfg* cfg, const pw_affinity_cfg* acfg,
-                            uint8_t* critical, int32_t* bins, pw_stream_t stream);
+                            uint8_t* critical, int32_t* bins, int32_t* unique,
+                            pw_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------
  * pw_cache_step [SUB]: one decode step of an expert cache (Quality-First = PW_POLICY_THRESHOLD
@@ -273,6 +278,12 @@ pw_status pw_cache_step(const float* logits, int32_t* idx, const float* gate, in
 
 /* ---------------------------------------------------------------------------------------
  * pw_moe_workspace_bytes: device workspace needed by pw_moe_anyprec_forward (0 on bad args).
+ * After a forward the workspace begins with the grouping it ran on, each region at a 256-byte
+ * boundary: counts int32[E] (assignments per expert), offsets int32[E+1] (exclusive prefix
+ * sums), perm int32[T*k] (grouped position -> assignment t*k + slot, ascending within an
+ * expert), inv int32[T*k] (assignment -> grouped position, -1 for an invalid expert id),
+ * active int32[E] (experts with work, ascending; the first meta[0] are valid), meta int32[8]
+ * (meta[0] = active experts).  The rest is scratch of no fixed layout.
  * ------------------------------------------------------------------------------------- */
 size_t pw_moe_workspace_bytes(int T, int k, int E, int H, int I);
 

@@ -109,11 +109,12 @@ def test_tc_switch_is_host_only(libpw):
 
 def test_workspace_holds_tensor_core_operands(libpw):
     # the workspace has room for both FFN paths: among the rest, the fp16 operands of the
-    # tensor-core path, one row per padded position (each active expert's rows rounded up to 16)
+    # tensor-core path, one row per padded position (each active expert's rows rounded up to 16):
+    # x (H columns) and h as hi and lo parts (2 I columns)
     for T, k, E, H, I in [(1, 2, 8, 4096, 14336), (64, 8, 64, 3584, 2560), (4, 2, 8, 256, 512),
                           (512, 10, 512, 2048, 512)]:
         ws = B.pw_moe_workspace_bytes(T, k, E, H, I)
         tk = T * k
         rows_pad = tk + 15 * min(E, tk)
-        assert ws >= 2 * rows_pad * (H + I) + 4 * tk * H * 8
+        assert ws >= 2 * rows_pad * (H + 2 * I) + 4 * tk * H * 8
         assert ws % 256 == 0

@@ -37,13 +37,17 @@ def _affinity_gpu(torch, lo, io, go, k, critical_n, nb, w, low):
     l_d, i_d, g_d = t(lo), t(io), t(go)
     crit = torch.empty((E,), dtype=torch.uint8, device=dev)
     bins = torch.empty((T,), dtype=torch.int32, device=dev)
+    uniq = torch.full((2,), -1, dtype=torch.int32, device=dev)
     cfg = B.pw_route_cfg(k=k, renorm=0, policy=0, threshold=0.15, critical_n=critical_n)
     acfg = B.pw_affinity_cfg(num_bins=nb, low_bins=low, bin_width=w)
     st = torch.cuda.current_stream().cuda_stream
     B.check(B.pw_affinity_remap(l_d.data_ptr(), i_d.data_ptr(), g_d.data_ptr(), T, E, cfg, acfg,
-                                crit.data_ptr(), bins.data_ptr(), st), "pw_affinity_remap")
+                                crit.data_ptr(), bins.data_ptr(), uniq.data_ptr(), st),
+            "pw_affinity_remap")
     assert B.pw_get_status(st) == B.PW_OK
-    return i_d.cpu().numpy(), crit.cpu().numpy(), bins.cpu().numpy()
+    i2 = i_d.cpu().numpy()
+    assert uniq.cpu().tolist() == [len(np.unique(io)), len(np.unique(i2))]
+    return i2, crit.cpu().numpy(), bins.cpu().numpy()
 
 
 @pytest.mark.parametrize("name,T", [("qwen2_57b_a14b", 8), ("qwen2_57b_a14b", 32),

@@ -159,10 +159,14 @@ def _remap_gpu(torch, dev, lo, io, go, k, critical_n):
     t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
     l_d, i_d, g_d = t(lo), t(io), t(go)
     crit = torch.empty((E,), dtype=torch.uint8, device=dev)
+    uniq = torch.full((2,), -1, dtype=torch.int32, device=dev)
     cfg = B.pw_route_cfg(k=k, renorm=0, policy=0, threshold=0.15, critical_n=critical_n)
     B.check(B.pw_remap(l_d.data_ptr(), i_d.data_ptr(), g_d.data_ptr(), T, E, cfg,
-                       crit.data_ptr(), _stream(torch)))
-    return i_d.cpu().numpy(), crit.cpu().numpy()
+                       crit.data_ptr(), uniq.data_ptr(), _stream(torch)))
+    i2 = i_d.cpu().numpy()
+    # the distinct experts before / after the rewrite (the experts the FFN reads)
+    assert uniq.cpu().tolist() == [len(np.unique(io)), len(np.unique(i2))]
+    return i2, crit.cpu().numpy()
 
 
 @pytest.mark.parametrize("T", [8, 32, 64])
