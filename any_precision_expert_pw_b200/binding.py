@@ -11,7 +11,9 @@ import ctypes
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libpw.so")
+# PW_LIB_VARIANT=debug loads the debug build (device bounds checks, PW_ERR_BOUNDS)
+LIB_PATH = os.path.join(HERE, "libpw_debug.so" if os.environ.get("PW_LIB_VARIANT") == "debug"
+                        else "libpw.so")
 
 PW_OK = 0
 PW_ERR_INVALID_ARG = 1
@@ -21,6 +23,7 @@ PW_ERR_NOT_RESIDENT = 4
 PW_ERR_TIMEOUT = 5
 PW_ERR_BAD_EXPERT = 6
 PW_ERR_BAD_BITS = 7
+PW_ERR_BOUNDS = 8
 
 PW_MOD_GATE_UP = 0
 PW_MOD_DOWN = 1

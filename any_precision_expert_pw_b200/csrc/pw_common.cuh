@@ -35,6 +35,20 @@ __device__ int g_status = 0;
 
 __device__ __forceinline__ void set_status(int code) { atomicCAS(&g_status, 0, code); }
 
+// Device bounds checks of the debug build (compiled with PW_DEBUG, libpw_debug.so): a global
+// address derived from runtime data (expert ids, counts, offsets, positions, block descriptors)
+// is checked against its buffer before the access; a failed check records PW_ERR_BOUNDS and the
+// access is skipped -- the kernel never traps.  In the normal build the checks compile away.
+#ifdef PW_DEBUG
+__device__ __forceinline__ bool pw_check(bool ok) {
+  if (!ok) set_status(PW_ERR_BOUNDS);
+  return ok;
+}
+#define PW_CHECK(cond) (::pw::pw_check(static_cast<bool>(cond)))
+#else
+#define PW_CHECK(cond) true
+#endif
+
 // Bound on every spin wait: a wait that has not completed after g_wait_limit_ns nanoseconds of
 // global time records PW_ERR_TIMEOUT and gives up.  Normal waits finish in microseconds; the
 // default is 2 s, and pw_set_wait_limit_ns() (a test hook) shortens it.

@@ -133,6 +133,8 @@ struct ModeParams {
   long long ld_act;   // elements between rows of act
   const int32_t* act_map;  // non-null: grouped position pos reads row act_map[pos] / act_div
   int act_div;             // (gate_up: the token of the assignment); null: row = pos
+  int act_rows;            // rows of act (bounds of the debug build)
+  int out_rows;            // grouped positions (T * k)
   int ld_out;
   __half* hout;         // gate_up: the down projection's activations [pos][ld_hout], xpos order
   long long ld_hout;
@@ -185,7 +187,12 @@ __device__ __forceinline__ Desc resolve(const Params& p, const ModeParams* mps, 
   d.a = a;
   d.pair = rem / mp.kslices;
   d.ks = rem - d.pair * mp.kslices;
-  const ExpertDesc x = p.xd[mode * p.E + a];
+  ExpertDesc x = p.xd[mode * p.E + a];
+  if (!PW_CHECK(a < p.E && x.pos0 >= 0 && x.te >= 0 && x.pos0 + x.te <= mp.out_rows)) {
+    x.valid = 0;  // an inconsistent grouping: nothing of this item is read or written
+    x.te = 0;
+    x.status = PW_ERR_BOUNDS;
+  }
   d.q = x.q;
   d.n = x.n;
   d.te = x.te;
@@ -688,7 +695,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
         if (!reuse) {
           for (int t = 0; t < ntok; ++t) {
             const int pos = cur.pos0 + ch + t;
-            const int r = mp.act_map ? mp.act_map[pos] / mp.act_div : pos;
+            int r = mp.act_map ? mp.act_map[pos] / mp.act_div : pos;
+            if (!PW_CHECK(r >= 0 && r < mp.act_rows)) r = 0;  // (debug build) read row 0
             arow[t] =
                 reinterpret_cast<const uint8_t*>(mp.act + static_cast<size_t>(r) * mp.ld_act);
           }
@@ -746,7 +754,8 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
           const size_t pos = static_cast<size_t>(it.pos0 + t);
           if (it.mode == MODE_GATE_UP) {
             store_h(mp.hout + pos * mp.ld_hout, it.pair * 32 + lane, 0.f);
-          } else {
+          } else if (PW_CHECK(pos < static_cast<size_t>(mp.out_rows) &&
+                              it.pair * kItemRows + 64 <= mp.ld_out)) {
             float* o = mp.out + it.ks * mp.out_slice + pos * mp.ld_out + it.pair * kItemRows;
             o[lane] = 0.f;
             o[32 + lane] = 0.f;
@@ -766,6 +775,7 @@ __global__ void __launch_bounds__(kThreads, 1) ffn_kernel(const Params p) {
             tb += rb[((w * NTP + t) * 2 + 1) * 32 + lane];
           }
           const size_t pos = static_cast<size_t>(it.pos0 + ch + t);
+          if (!PW_CHECK(pos < static_cast<size_t>(mp.out_rows))) continue;
           if (it.mode == MODE_GATE_UP) {
             // lane i < 16: gate rows of features 32P + i (row a) and 32P + 16 + i (row b);
             // lane i + 16: the matching up rows

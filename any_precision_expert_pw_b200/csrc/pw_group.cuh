@@ -32,6 +32,48 @@ __host__ __device__ __forceinline__ int pass_np(int count, int j) {
   return (m + 15) & ~15;
 }
 
+// Exclusive prefix sums of four counters over the threads of the CTA (blockDim.x <= 1024, a
+// multiple of 32), in thread order; every thread also gets the totals.  CTA-wide.
+__device__ __forceinline__ int4 block_scan4(int4 v, int4& total) {
+  __shared__ int4 wsum[32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int4 inc = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int x = __shfl_up_sync(0xffffffffu, inc.x, off), y = __shfl_up_sync(0xffffffffu, inc.y, off);
+    const int z = __shfl_up_sync(0xffffffffu, inc.z, off), w = __shfl_up_sync(0xffffffffu, inc.w, off);
+    if (lane >= off) {
+      inc.x += x;
+      inc.y += y;
+      inc.z += z;
+      inc.w += w;
+    }
+  }
+  if (lane == 31) wsum[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    int4 t = lane < nw ? wsum[lane] : make_int4(0, 0, 0, 0);
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, t.x, off), y = __shfl_up_sync(0xffffffffu, t.y, off);
+      const int z = __shfl_up_sync(0xffffffffu, t.z, off), w = __shfl_up_sync(0xffffffffu, t.w, off);
+      if (lane >= off) {
+        t.x += x;
+        t.y += y;
+        t.z += z;
+        t.w += w;
+      }
+    }
+    if (lane < nw) wsum[lane] = t;  // inclusive sums of the warp totals
+  }
+  __syncthreads();
+  const int4 before = warp ? wsum[warp - 1] : make_int4(0, 0, 0, 0);
+  total = wsum[nw - 1];
+  __syncthreads();  // wsum may be reused by the next call
+  return make_int4(before.x + inc.x - v.x, before.y + inc.y - v.y, before.z + inc.z - v.z,
+                   before.w + inc.w - v.w);
+}
+
 // Grouping, run by one CTA.  counts[E], offsets[E+1], perm[T*k] (grouped position ->
 // assignment), inv[T*k] (assignment -> grouped position, -1 for an invalid expert id),
 // active[E] (experts with work, ascending), meta[0] = number of active experts (0 when the page
@@ -64,30 +106,33 @@ __device__ __forceinline__ void group_block(const pw_page_table* __restrict__ pt
     eid[a] = static_cast<int16_t>(e);
   }
   __syncthreads();
-  if (tid == 0) {  // E <= 1024: a serial scan is a few hundred cycles
-    const bool bad = pt->blocks == nullptr || static_cast<unsigned>(layer) >= pt->num_layers ||
-                     static_cast<int>(pt->num_experts) != E ||
-                     (reinterpret_cast<uintptr_t>(pt->blocks) & 63) != 0;
+  // per expert (thread e): assignments, active or not, padded rows and tensor-core passes;
+  // their exclusive prefix sums give the offsets, the active index, the padded row base and
+  // the first pass of each expert (E <= blockDim.x)
+  const bool bad = pt->blocks == nullptr || static_cast<unsigned>(layer) >= pt->num_layers ||
+                   static_cast<int>(pt->num_experts) != E ||
+                   (reinterpret_cast<uintptr_t>(pt->blocks) & 63) != 0;
+  const int c = tid < E ? cnt[tid] : 0;
+  const int4 mine = make_int4(c, c > 0 ? 1 : 0, (c + 15) & ~15,
+                              bad ? 0 : (c + kPassTokens - 1) / kPassTokens);
+  int4 total;
+  const int4 ex = block_scan4(mine, total);
+  if (tid < E) {
+    off[tid] = ex.x;
+    act_pos[tid] = ex.y;
+    pb[tid] = ex.z;
+    for (int j = 0; j < mine.w; ++j) po.pass_tab[ex.w + j] = ex.y | (j << 16);
+  }
+  if (tid == 0) {
     if (bad) set_status(PW_ERR_INVALID_ARG);
-    int o = 0, na = 0, prow = 0, npass = 0;
-    for (int e = 0; e < E; ++e) {
-      off[e] = o;
-      act_pos[e] = na;
-      pb[e] = prow;
-      if (cnt[e] > 0 && !bad)
-        for (int j = 0; j * kPassTokens < cnt[e]; ++j) po.pass_tab[npass++] = na | (j << 16);
-      o += cnt[e];
-      prow += (cnt[e] + 15) & ~15;
-      na += (cnt[e] > 0);
-    }
-    off[E] = o;
-    act_pos[E] = na;
-    meta[0] = bad ? 0 : na;
-    meta[1] = o;
+    off[E] = total.x;
+    act_pos[E] = total.y;
+    meta[0] = bad ? 0 : total.y;
+    meta[1] = total.x;
     meta[2] = bad ? 1 : 0;
     meta[4] = 0;  // work counter of the FFN launch
-    meta[5] = npass;
-    meta[6] = prow;
+    meta[5] = total.w;
+    meta[6] = total.z;
   }
   __syncthreads();
   for (int e = tid; e < E; e += blockDim.x) {
@@ -189,10 +234,12 @@ __global__ void __launch_bounds__(256) stage_x_kernel(const uint16_t* __restrict
                                                       int vec, const int32_t* __restrict__ ptok,
                                                       const int32_t* __restrict__ pnn,
                                                       const int32_t* __restrict__ meta,
+                                                      int T, int rows_cap,
                                                       __half* __restrict__ XB) {
   griddep_wait();  // grouping of the launch before
   griddep_launch();
-  const int rows = meta[6];
+  int rows = meta[6];
+  if (!PW_CHECK(rows <= rows_cap)) rows = 0;
   const int g8 = H / 8;
   const size_t n_all = static_cast<size_t>(rows) * g8;
   for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_all;
@@ -202,6 +249,7 @@ __global__ void __launch_bounds__(256) stage_x_kernel(const uint16_t* __restrict
     const int tok = ptok[row];
     const int nn = pnn[row];
     const int np = nn >> 16, n = nn & 0xffff;
+    if (!PW_CHECK(tok < T && n < np && row - n + np <= rows)) continue;
     __half* dst = XB + static_cast<size_t>(row - n) * H + (c / kTcChunkCols) * np * kTcChunkCols +
                   ((c % kTcChunkCols) / 8) * np * 8 + n * 8;
     uint4 out = make_uint4(0u, 0u, 0u, 0u);
@@ -243,6 +291,7 @@ __global__ void combine_kernel(const float* __restrict__ O, const int32_t* __res
     for (int s = 0; s < k; ++s) {
       const int pos = inv[t * k + s];
       if (pos < 0 || bad) continue;
+      if (!PW_CHECK(static_cast<long long>(pos) * H < slice)) continue;
       float o = 0.0f;
       for (int j = 0; j < kslices; ++j) o += O[j * slice + static_cast<size_t>(pos) * H + r];
       acc = fmaf(gate[t * k + s], o, acc);

@@ -204,7 +204,11 @@ pw_status forward_args_status(const pw_page_table* pt_dev, int layer, int E,
 
 extern "C" {
 
-const char* pw_version(void) { return "libpw 0.1 (sm_100a)"; }
+#ifdef PW_DEBUG
+const char* pw_version(void) { return "libpw 0.2 (sm_100a, debug: device bounds checks)"; }
+#else
+const char* pw_version(void) { return "libpw 0.2 (sm_100a)"; }
+#endif
 
 const char* pw_status_string(pw_status s) {
   switch (s) {
@@ -216,6 +220,7 @@ const char* pw_status_string(pw_status s) {
     case PW_ERR_TIMEOUT: return "PW_ERR_TIMEOUT";
     case PW_ERR_BAD_EXPERT: return "PW_ERR_BAD_EXPERT";
     case PW_ERR_BAD_BITS: return "PW_ERR_BAD_BITS";
+    case PW_ERR_BOUNDS: return "PW_ERR_BOUNDS";
   }
   return "PW_ERR_UNKNOWN";
 }
@@ -305,7 +310,8 @@ pw_status pw_moe_anyprec_forward(const pw_page_table* pt_dev, int layer, int E,
       if (launch_dependent(pw::stage_x_kernel, dim3(grid), dim3(256), 0, st, x_bf16, H, vec,
                            static_cast<const int32_t*>(po.ptok),
                            static_cast<const int32_t*>(po.pnn),
-                           static_cast<const int32_t*>(meta), XB) != PW_OK)
+                           static_cast<const int32_t*>(meta), T,
+                           static_cast<int>(rows_pad), XB) != PW_OK)
         return PW_ERR_CUDA;
     }
     pw::k5::Params q;
@@ -379,6 +385,8 @@ pw_status pw_moe_anyprec_forward(const pw_page_table* pt_dev, int layer, int E,
   gu.ld_act = w.ldx;
   gu.act_map = perm;  // grouped position -> assignment t*k+slot -> token row of X
   gu.act_div = k;
+  gu.act_rows = T;
+  gu.out_rows = TK;
   gu.hout = Hb;
   gu.ld_hout = w.ldh;
   gu.out = nullptr;
@@ -398,6 +406,8 @@ pw_status pw_moe_anyprec_forward(const pw_page_table* pt_dev, int layer, int E,
   dn.ld_act = w.ldh;
   dn.act_map = nullptr;
   dn.act_div = 1;
+  dn.act_rows = TK;
+  dn.out_rows = TK;
   dn.hout = nullptr;
   dn.ld_hout = 0;
   dn.out = O;

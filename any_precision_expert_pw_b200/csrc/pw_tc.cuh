@@ -183,6 +183,13 @@ __device__ __forceinline__ Desc resolve(const Params& p, int item, int npass) {
   d.lut = bits_ok ? b->lut[d.q] : nullptr;
   d.valid = bits_ok && shape_ok && resident;
   d.status = !shape_ok ? PW_ERR_INVALID_ARG : (!resident ? PW_ERR_NOT_RESIDENT : PW_ERR_BAD_BITS);
+  // (debug build) the pass lies inside the grouping: positions and padded rows
+  if (!PW_CHECK(a < p.E && d.pos0 >= 0 && d.pos0 + d.te <= p.meta[1] &&
+                d.prow0 + d.np <= p.meta[6])) {
+    d.valid = 0;
+    d.te = 0;
+    d.status = PW_ERR_BOUNDS;
+  }
   return d;
 }
 

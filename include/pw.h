@@ -56,8 +56,11 @@ typedef enum {
   PW_ERR_NOT_RESIDENT = 4, /* device: a used block's page state is not PW_PAGE_GPU      */
   PW_ERR_TIMEOUT = 5,      /* device: a bounded wait gave up                            */
   PW_ERR_BAD_EXPERT = 6,   /* device: an expert id outside [0, E)                        */
-  PW_ERR_BAD_BITS = 7      /* device: committed bitwidth outside [min_bits, parent_bits]
+  PW_ERR_BAD_BITS = 7,     /* device: committed bitwidth outside [min_bits, parent_bits]
                               or its LUT missing                                        */
+  PW_ERR_BOUNDS = 8        /* device, debug build (libpw_debug.so) only: an address derived
+                              from runtime data fell outside its buffer; the access was
+                              skipped                                                   */
 } pw_status;
 
 enum { PW_MOD_GATE_UP = 0, PW_MOD_DOWN = 1 };

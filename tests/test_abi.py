@@ -21,6 +21,19 @@ def test_header_and_binding_agree(libpw):
         assert hasattr(libpw, name), name
 
 
+def test_debug_build_exports_the_same_functions(libpw):
+    # libpw_debug.so: the same C ABI with device bounds checks (PW_ERR_BOUNDS)
+    path = os.path.join(os.path.dirname(B.LIB_PATH), "libpw_debug.so")
+    dbg = ctypes.CDLL(path)
+    for name in _declared():
+        assert hasattr(dbg, name), name
+    dbg.pw_version.restype = ctypes.c_char_p
+    assert b"debug" in dbg.pw_version() and b"sm_100a" in dbg.pw_version()
+    dbg.pw_status_string.restype = ctypes.c_char_p
+    assert dbg.pw_status_string(B.PW_ERR_BOUNDS) == b"PW_ERR_BOUNDS"
+    assert B.pw_status_string(B.PW_ERR_BOUNDS) == "PW_ERR_BOUNDS"
+
+
 def test_status_strings_and_version(libpw):
     assert B.pw_status_string(B.PW_OK) == "PW_OK"
     assert B.pw_status_string(B.PW_ERR_BAD_BITS) == "PW_ERR_BAD_BITS"
