@@ -13,6 +13,7 @@ PKG = os.path.dirname(HERE)
 ROOT = os.path.dirname(PKG)
 OUT = os.path.join(PKG, "libpw.so")
 OUT_DEBUG = os.path.join(PKG, "libpw_debug.so")
+OUT_CEILING = os.path.join(PKG, "decode_ceiling")
 SOURCES = [os.path.join(HERE, "pw_lib.cu")]
 DEPS = [os.path.join(HERE, f) for f in os.listdir(HERE) if f.endswith((".cu", ".cuh"))] + [
     os.path.join(ROOT, "include", "pw.h")]
@@ -55,6 +56,17 @@ def build(force: bool = False, verbose_ptxas: bool = False, debug: bool = True) 
     return OUT
 
 
+def build_ceiling() -> str:
+    """The decode-ceiling measurement program (decode_ceiling.cu, a standalone executable)."""
+    subprocess.run([nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo",
+                    "-std=c++17", "-I", os.path.join(ROOT, "include"), "-I", HERE, "-o",
+                    OUT_CEILING, os.path.join(HERE, "decode_ceiling.cu")], check=True)
+    return OUT_CEILING
+
+
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose_ptxas="-v" in sys.argv)
-    print(OUT)
+    if "--ceiling" in sys.argv:
+        print(build_ceiling())
+    else:
+        build(force="--force" in sys.argv, verbose_ptxas="-v" in sys.argv)
+        print(OUT)
