@@ -92,6 +92,7 @@ __device__ __forceinline__ void group_block(const pw_page_table* __restrict__ pt
   __shared__ int act_pos[PW_MAX_EXPERTS + 1];
   __shared__ int pb[PW_MAX_EXPERTS];
   __shared__ int16_t eid[kMaxAssign];
+  __shared__ int run[PW_MAX_EXPERTS];
   const int tid = threadIdx.x;
   for (int e = tid; e < E; e += blockDim.x) cnt[e] = 0;
   __syncthreads();
@@ -146,14 +147,32 @@ __device__ __forceinline__ void group_block(const pw_page_table* __restrict__ pt
     }
   }
   if (tid == 0) offsets[E] = off[E];
-  for (int a = tid; a < TK; a += blockDim.x) {
-    const int e = eid[a];
+  // rank of each assignment among its expert's (ascending a): chunks of blockDim assignments in
+  // order; inside a warp the peers of an expert come from one match, and the warps of a chunk
+  // take their bases from run[e] one after the other
+  const int lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+  for (int e = tid; e < E; e += blockDim.x) run[e] = 0;
+  __syncthreads();
+  for (int c0 = 0; c0 < TK; c0 += blockDim.x) {
+    const int a = c0 + tid;
+    const int e = a < TK ? eid[a] : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int leader = __ffs(peers) - 1;
+    int base = 0;
+    for (int w = 0; w < nw; ++w) {
+      if (warp == w && e >= 0 && lane == leader) {
+        base = run[e];
+        run[e] = base + __popc(peers);
+      }
+      __syncthreads();
+    }
+    base = __shfl_sync(0xffffffffu, base, leader);
+    if (a >= TK) continue;
     if (e < 0) {
       inv[a] = -1;
       continue;
     }
-    int r = 0;
-    for (int b = 0; b < a; ++b) r += (eid[b] == e);
+    const int r = base + __popc(peers & ((1u << lane) - 1u));
     const int pos = off[e] + r;
     perm[pos] = a;
     inv[a] = pos;

@@ -26,6 +26,10 @@ __device__ __forceinline__ double bf16hi(uint32_t v) {
 // (float64 exp has a long latency): the selected experts' probabilities are read back from the
 // lane that holds them.  PL = elements per lane (E <= 32 * PL), so the code is no larger than
 // E needs (a cold kernel fetches every instruction it runs from memory).
+// float64 exp behind a call, so the PL exponentials of topk_warp share one copy of its code
+// (a cold kernel fetches every instruction it runs from memory).
+__device__ __noinline__ double exp_f64(double v) { return exp(v); }
+
 template <int PL>
 __device__ __forceinline__ void topk_warp(const float* l, int E, int k, int renorm,
                                           int32_t* __restrict__ idx_out,
@@ -47,7 +51,8 @@ __device__ __forceinline__ void topk_warp(const float* l, int E, int k, int reno
   for (int i = 0; i < PL; ++i) {
     ex[i] = 0.0;
     if (lane + 32 * i < E) {
-      ex[i] = exp(static_cast<double>(v[i]) - static_cast<double>(mx));
+      ex[i] = PL > 2 ? exp_f64(static_cast<double>(v[i]) - static_cast<double>(mx))
+                     : exp(static_cast<double>(v[i]) - static_cast<double>(mx));
       z += ex[i];
     }
   }
@@ -267,16 +272,24 @@ __global__ void __launch_bounds__(256) substitute_kernel(
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
-  int cur[PW_MAX_TOPK];
-  bool bad = false;
-  for (int j = 0; j < k; ++j) {
-    cur[j] = idx[static_cast<size_t>(t) * k + j];
-    bad |= (cur[j] < 0 || cur[j] >= E);
+  // lane j < k reads slot j (id, gate, residency of the routed expert), so the token's slots
+  // cost two dependent round trips to memory instead of two per slot
+  int my_e = 0;
+  float my_g = 0.0f;
+  int my_res = 0;
+  if (lane < k) {
+    my_e = idx[static_cast<size_t>(t) * k + lane];
+    my_g = gate[static_cast<size_t>(t) * k + lane];
   }
+  const bool bad = __any_sync(0xffffffffu, lane < k && (my_e < 0 || my_e >= E));
   if (bad) {  // ids out of range: leave the token untouched
     if (lane == 0) set_status(PW_ERR_BAD_EXPERT);
     return;
   }
+  if (lane < k) my_res = resident[my_e] ? 1 : 0;
+  const uint32_t res_slots = __ballot_sync(0xffffffffu, my_res != 0);  // bit s: slot s resident
+  int cur[PW_MAX_TOPK];
+  for (int j = 0; j < k; ++j) cur[j] = __shfl_sync(0xffffffffu, my_e, j);
   WarpRow<PL> row;
   load_row(logits + static_cast<size_t>(t) * E, E, row);
   uint32_t res = 0;
@@ -289,9 +302,9 @@ __global__ void __launch_bounds__(256) substitute_kernel(
   double sub = 0.0, tot = 0.0;
   uint8_t act[PW_MAX_TOPK];
   for (int s = 0; s < k; ++s) {
-    const float g = gate[static_cast<size_t>(t) * k + s];
+    const float g = __shfl_sync(0xffffffffu, my_g, s);
     tot += static_cast<double>(g);
-    if (resident[cur[s]]) {
+    if ((res_slots >> s) & 1u) {  // the expert routed to slot s (never rewritten before s)
       act[s] = PW_ACT_HIT;
       continue;
     }
