@@ -35,11 +35,13 @@
 //                          completion to the barrier that frees its B buffer, each chunk's to the
 //                          one that frees its A buffer.
 // The down projection's activations h are fp32 results of the gate_up epilogue; they are held as
-// hi = fp16(h) and lo = fp16(h - hi) and multiplied as two operands into the same accumulator,
-// so the products keep h to about 22 bits (a single fp16 rounding of h, 2^-11 relative, leaves
-// the whole output of a large batch at the edge of the parity bar).  A pass of more than 32
-// tokens is split into two sub-passes of 32 + the rest (MMA N of 32 and np - 32), each of
-// whose hi and lo blocks of a chunk fit one B buffer.
+// hi = fp16(h) and lo = fp16(h - hi), so the products keep h to about 22 bits (a single fp16
+// rounding of h, 2^-11 relative, leaves the whole output of a large batch at the edge of the
+// parity bar).  A down operand block stacks, per 8-column K group, the nps hi rows and then the
+// nps lo rows: one MMA of N = 2 nps per K step writes the hi products to accumulator columns
+// [0, nps) and the lo products to [nps, 2 nps), and the epilogue adds the two.  A pass of more
+// than 32 tokens is split into two sub-passes of 32 + the rest (accumulator columns 64 sp ..),
+// so that a sub-pass's block of a chunk fits one B buffer.
 // The decode table pairs rows r and r + 64 of the item: the 32-bit slot at byte 256v + 4r
 // (r < 64) holds (LUT_r[v], LUT_{r+64}[v]).  A warp's 32 rows are 32 consecutive r mod 64, so
 // its gathers hit 32 different banks, the slot address is one byte permute of the code byte,
@@ -65,10 +67,12 @@ constexpr int kPlaneWarp = 20;
 constexpr int kOperandWarp = 21;
 constexpr int kMmaWarp = 22;
 constexpr int kThreads = 23 * 32;
-// tensor memory: two accumulators of up to 64 fp32 columns, then two A buffers of 128 columns
-// (128 rows x 256 fp16); the allocation is the next power of two, 512
+// tensor memory: two accumulators of 128 fp32 columns (a gate_up pass uses np of them, a down
+// pass 2 np: the products with h's hi parts and with its lo parts side by side), then two A
+// buffers of 128 columns (128 rows x 256 fp16): 512 columns
 constexpr int kTmemCols = 512;
-constexpr int kTmemA = 2 * kPass;
+constexpr int kAccCols = 2 * kPass;
+constexpr int kTmemA = 2 * kAccCols;
 constexpr int kACols = kChunkCols / 2;
 constexpr int kPlaneStages = 3;
 constexpr int kDescRing = 8;
@@ -248,6 +252,18 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+  uint32_t r[8];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   if (*abort_flag) return false;
   if (!mbar_wait(bar, parity, abort_flag)) {
@@ -413,7 +429,8 @@ __device__ __forceinline__ void prefetch_item(const Params& p, const Desc& d) {
 // Place of h element (token n of the pass, feature f) in the down operand staging, relative to
 // the pass's first padded row (2 I fp16 per padded row): sub-pass sp = n / 32 of a pass of
 // more than 32 tokens (sub-pass 0 then holds 32 rows), then per 256-column chunk one block of
-// np_s rows hi followed by np_s rows lo, each in the MMA's K-major core-matrix order.
+// 2 np_s rows in the MMA's K-major core-matrix order: rows [0, np_s) the hi parts of the
+// sub-pass's tokens, rows [np_s, 2 np_s) their lo parts.
 struct HPlace {
   size_t hi, lo;
 };
@@ -423,8 +440,9 @@ __device__ __forceinline__ HPlace h_place(int np, int I, int n, int f) {
   const int nn = n - 32 * sp;
   const int c = f / kChunkCols, cc = min(kChunkCols, I - c * kChunkCols);
   const size_t blk = static_cast<size_t>(sp) * 64 * I + static_cast<size_t>(c) * 2 * nps * kChunkCols;
-  const size_t in = static_cast<size_t>((f % kChunkCols) / 8) * nps * 8 + nn * 8 + (f % 8);
-  return {blk + in, blk + static_cast<size_t>(nps) * cc + in};
+  const size_t in = static_cast<size_t>((f % kChunkCols) / 8) * 2 * nps * 8 + nn * 8 + (f % 8);
+  (void)cc;
+  return {blk + in, blk + in + static_cast<size_t>(nps) * 8};
 }
 
 // Epilogue of one item, warp j (rows 32j.. of the accumulator).  gate_up: lanes 0-15 hold the
@@ -436,9 +454,9 @@ __device__ __forceinline__ void epilogue(const Desc& d, const ModeParams& mp, in
   const int tile = d.mb * kTiles + j;
   const uint32_t lane_addr = tmem_acc + (static_cast<uint32_t>(j * 32) << 16);
   for (int c0 = 0; c0 < d.np; c0 += 16) {
-    float v[16];
-    tmem_ld16(lane_addr + c0, v);
     if (d.mode == MODE_GATE_UP) {
+      float v[16];
+      tmem_ld16(lane_addr + c0, v);
       const int f = tile * 16 + (lane & 15);
       // the down operand has I = mp.half columns
       __half* base = mp.hout + static_cast<size_t>(d.prow0) * 2 * mp.half;
@@ -455,11 +473,23 @@ __device__ __forceinline__ void epilogue(const Desc& d, const ModeParams& mp, in
         }
       }
     } else {
+      // tokens c0 .. c0 + 15 lie in one sub-pass sp: their hi products at accumulator columns
+      // 64 sp + (c0 - 32 sp) .., their lo products nps columns further
+      const int sp = (d.np > 32 && c0 >= 32) ? 1 : 0;
+      const int nps = d.np > 32 ? (sp ? d.np - 32 : 32) : d.np;
       float* base = mp.out + d.ks * mp.out_slice + static_cast<size_t>(d.pos0) * mp.ld_out +
                     tile * 32 + lane;
 #pragma unroll
-      for (int n = 0; n < 16; ++n)
-        if (c0 + n < d.te) base[static_cast<size_t>(c0 + n) * mp.ld_out] = v[n];
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t col = 64 * sp + (c0 - 32 * sp) + 8 * h;
+        float a[8], b[8];
+        tmem_ld8(lane_addr + col, a);
+        tmem_ld8(lane_addr + col + nps, b);
+#pragma unroll
+        for (int n = 0; n < 8; ++n)
+          if (c0 + 8 * h + n < d.te)
+            base[static_cast<size_t>(c0 + 8 * h + n) * mp.ld_out] = a[n] + b[n];
+      }
     }
   }
 }
@@ -642,7 +672,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ffn_kernel(const Params p) {
         const uint32_t acc = va & 1;
         if (!wait_bar(&acc_empty[acc], ((va >> 1) & 1) ^ 1, abort_flag)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * kPass;
+        const uint32_t d_tmem = tmem_base + acc * kAccCols;
         const int W = p.m[d.mode].cols / 32;
         const bool down = d.mode == MODE_DOWN;
         const int nsp = down && d.np > 32 ? 2 : 1;
@@ -665,17 +695,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ffn_kernel(const Params p) {
                            smem_desc(b_addr + s * 2 * d.np * 16, d.np * 16, 128), idesc,
                            (c > d.c0 || s > 0) ? 1u : 0u);
             } else {
-              // sub-pass sp: tokens 32 sp .. of the pass, accumulator columns 32 sp ..; its hi
-              // block then its lo block, into the same accumulator
+              // sub-pass sp: tokens 32 sp .. of the pass; N = 2 nps rows of B (hi, then lo)
+              // into accumulator columns 64 sp .. 64 sp + 2 nps
               const int nps = nsp == 2 ? (sp ? d.np - 32 : 32) : d.np;
-              const uint32_t idesc = instr_desc(nps);
-              for (int part = 0; part < 2; ++part) {
-                const uint32_t pb = b_addr + part * nps * cc * 2;
-                for (int s = 0; s < ksteps; ++s)
-                  mma_f16_ts(d_tmem + 32 * sp, a_tmem + 8 * s,
-                             smem_desc(pb + s * 2 * nps * 16, nps * 16, 128), idesc,
-                             (c > d.c0 || part > 0 || s > 0) ? 1u : 0u);
-              }
+              const int n2 = 2 * nps;
+              const uint32_t idesc = instr_desc(n2);
+              for (int s = 0; s < ksteps; ++s)
+                mma_f16_ts(d_tmem + 64 * sp, a_tmem + 8 * s,
+                           smem_desc(b_addr + s * 2 * n2 * 16, n2 * 16, 128), idesc,
+                           (c > d.c0 || s > 0) ? 1u : 0u);
+              (void)cc;
             }
             mma_commit(&b_empty[b]);
           }
@@ -751,7 +780,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ffn_kernel(const Params p) {
         const uint32_t acc = (va - 1) & 1;
         if (!warp_wait(&acc_full[acc], ((va - 1) >> 1) & 1, abort_flag)) break;
         tc_fence_after();
-        epilogue(prev, p.m[prev.mode], ew, lane, tmem_base + acc * kPass);
+        epilogue(prev, p.m[prev.mode], ew, lane, tmem_base + acc * kAccCols);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[acc]);
@@ -769,7 +798,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ffn_kernel(const Params p) {
       const uint32_t acc = (va - 1) & 1;
       if (warp_wait(&acc_full[acc], ((va - 1) >> 1) & 1, abort_flag)) {
         tc_fence_after();
-        epilogue(prev, p.m[prev.mode], ew, lane, tmem_base + acc * kPass);
+        epilogue(prev, p.m[prev.mode], ew, lane, tmem_base + acc * kAccCols);
         tc_fence_before();
         if (prev.mode == MODE_GATE_UP) {
           __threadfence();
