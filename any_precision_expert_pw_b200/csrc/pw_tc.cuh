@@ -688,24 +688,21 @@ __global__ void __launch_bounds__(kThreads, 1) tc_ffn_kernel(const Params p) {
             if (!(ok = wait_bar(&b_full[b], (g >> 1) & 1, abort_flag))) break;
             tc_fence_after();
             const uint32_t b_addr = smem_u32(smem + kOffB + b * kBBytes);
-            if (!down) {
-              const uint32_t idesc = instr_desc(d.np);
-              for (int s = 0; s < ksteps; ++s)  // 8 columns of A per step
-                mma_f16_ts(d_tmem, a_tmem + 8 * s,
-                           smem_desc(b_addr + s * 2 * d.np * 16, d.np * 16, 128), idesc,
-                           (c > d.c0 || s > 0) ? 1u : 0u);
-            } else {
-              // sub-pass sp: tokens 32 sp .. of the pass; N = 2 nps rows of B (hi, then lo)
-              // into accumulator columns 64 sp .. 64 sp + 2 nps
-              const int nps = nsp == 2 ? (sp ? d.np - 32 : 32) : d.np;
-              const int n2 = 2 * nps;
-              const uint32_t idesc = instr_desc(n2);
-              for (int s = 0; s < ksteps; ++s)
-                mma_f16_ts(d_tmem + 64 * sp, a_tmem + 8 * s,
-                           smem_desc(b_addr + s * 2 * n2 * 16, n2 * 16, 128), idesc,
-                           (c > d.c0 || s > 0) ? 1u : 0u);
-              (void)cc;
-            }
+            // the rows of B this block multiplies (gate_up: the pass's np tokens; down: sub-pass
+            // sp's nps tokens, hi rows then lo rows) and where they accumulate (down: columns
+            // 64 sp .., hi products then lo products)
+            const int nps = down ? (nsp == 2 ? (sp ? d.np - 32 : 32) : d.np) : d.np;
+            const int nb = down ? 2 * nps : d.np;
+            const uint32_t idesc = instr_desc(nb);
+            const uint32_t dt = d_tmem + (down ? 64 * sp : 0);
+            // descriptor of K step 0; step s starts 2 K groups (2 nb 16 bytes) further on, a
+            // plain add to the address field (shared-memory addresses stay below 2^18)
+            const uint64_t bd0 = smem_desc(b_addr, nb * 16, 128);
+            const uint64_t bstep = static_cast<uint64_t>((2 * nb * 16) >> 4);
+            mma_f16_ts(dt, a_tmem, bd0, idesc, c > d.c0 ? 1u : 0u);
+            for (int s = 1; s < ksteps; ++s)  // 8 columns of A per step
+              mma_f16_ts(dt, a_tmem + 8 * s, bd0 + s * bstep, idesc, 1u);
+            (void)cc;
             mma_commit(&b_empty[b]);
           }
           if (ok) mma_commit(&ab_empty[ab]);  // the chunk's A buffer is read
