@@ -85,6 +85,14 @@ struct Workspace {
   int ldx, ldh;
 };
 
+// Most k-slices either FFN path splits a down projection of I columns into (the CUDA-core
+// path's rule and choose_kslices both stay within it): at most kMaxKSlices, at least two
+// 512-column stages per slice.
+int max_kslices(int I) {
+  const int nst = (I + pw::k4::kStageCols - 1) / pw::k4::kStageCols;
+  return std::min(pw::k4::kMaxKSlices, std::max(1, nst / 2));
+}
+
 Workspace ws_layout(int T, int k, int E, int H, int I) {
   Workspace w;
   const size_t TK = static_cast<size_t>(T) * k;
@@ -107,7 +115,7 @@ Workspace ws_layout(int T, int k, int E, int H, int I) {
   w.done = take(4 * static_cast<size_t>(E));  // gate_up tiles finished per active expert
   w.X = take(2 * static_cast<size_t>(T) * w.ldx);
   w.Hbuf = take(2 * TK * w.ldh);
-  w.O = take(4 * TK * H * static_cast<size_t>(pw::k4::kMaxKSlices));
+  w.O = take(4 * TK * H * static_cast<size_t>(max_kslices(I)));
   w.xd = take(sizeof(pw::k4::ExpertDesc) * 2 * static_cast<size_t>(E));
   // tensor-core path: each active expert's rows padded to a multiple of 16
   const size_t rows_pad = TK + 15 * std::min<size_t>(E, TK);

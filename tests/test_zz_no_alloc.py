@@ -17,9 +17,10 @@ pytestmark = pytest.mark.gpu
 
 # (shape, T, pw_set_tc_min_tokens value): the CUDA-core path (scaled Mixtral-shaped layer,
 # 16 assignments over 8 experts) and the tensor-core path (forced), the Mixtral-shaped layer at
-# full size and batch 16 among them (its scratch need is close to the array's size)
+# full size and batch 16 among them (its scratch need is close to the array's size), and the
+# Qwen1.5-shaped layer at batch 64 (the tensor-core path by default, several experts per CTA)
 CASES = [("mixtral_scaled", 8, None), ("mixtral_scaled", 8, 0), ("mixtral_8x7b", 16, None),
-         ("mixtral_8x7b", 16, 0)]
+         ("mixtral_8x7b", 16, 0), ("qwen15_moe_a2.7b", 64, None)]
 
 
 def _cfg(name):
