@@ -219,15 +219,23 @@ __device__ __forceinline__ ExpertDesc expert_desc(const pw_page_table* pt, int l
   x.q = b->committed_bits;
   // planes held per (tile, stage) run on the device: all parent_bits, or a paged-in prefix
   x.n = b->stored_bits ? b->stored_bits : b->parent_bits;
+  // every LUT pointer a committed bitwidth can select, read with the other fields (one round
+  // trip to memory rather than a second one that waits for the bitwidth)
+  const uint16_t* lq = nullptr;
+#pragma unroll
+  for (int q = PW_MIN_BITS; q <= PW_MAX_BITS; ++q) {
+    const uint16_t* l = b->lut[q];
+    if (x.q == q) lq = l;
+  }
   const bool bits_ok = x.q >= b->min_bits && x.q <= x.n && x.n <= b->parent_bits &&
-                       x.q >= PW_MIN_BITS && x.q <= PW_MAX_BITS && b->lut[x.q] != nullptr &&
+                       x.q >= PW_MIN_BITS && x.q <= PW_MAX_BITS && lq != nullptr &&
                        b->planes != nullptr;
   const int want_layout = mode == MODE_GATE_UP ? PW_LAYOUT_TILED_GATE_UP : PW_LAYOUT_TILED_DOWN;
   const bool shape_ok = static_cast<int>(b->rows) == rows && static_cast<int>(b->cols) == cols &&
                         b->layout == want_layout;
   const bool resident = b->state == PW_PAGE_GPU;
   x.planes = b->planes;
-  x.lut = bits_ok ? b->lut[x.q] : nullptr;
+  x.lut = bits_ok ? lq : nullptr;
   x.tile_words = static_cast<long long>(x.n) * kTileRows * (cols / 32);
   x.valid = bits_ok && shape_ok && resident;
   x.status = !shape_ok ? PW_ERR_INVALID_ARG : (!resident ? PW_ERR_NOT_RESIDENT : PW_ERR_BAD_BITS);

@@ -12,6 +12,7 @@ constexpr int kGroupThreads = 1024;
 constexpr int kMaxAssign = 8192;  // T * k handled by the single-CTA grouping step
 constexpr int kPassTokens = 64;   // tokens of one expert per tensor-core pass (MMA N <= 64)
 constexpr int kTcChunkCols = 256; // K columns per tensor-core pipeline step (operand chunk)
+constexpr int kEarlyDescExperts = 64;  // setup reads every expert's blocks before grouping
 
 // What the tensor-core FFN needs beyond the plain grouping.  Each expert's tokens are split
 // into passes of up to kPassTokens; a pass of m tokens is padded to np = m rounded up to 16
@@ -79,7 +80,9 @@ __device__ __forceinline__ int4 block_scan4(int4 v, int4& total) {
 // active[E] (experts with work, ascending), meta[0] = number of active experts (0 when the page
 // table does not match (layer, E)), meta[1] = number of valid assignments, meta[2] = 1 for a
 // mismatched table, meta[4] = 0 (the FFN launch's work counter); and the PassOut arrays.
-__device__ __forceinline__ void group_block(const pw_page_table* __restrict__ pt, int layer,
+// Returns, to thread e < E, expert e's exclusive scan values: .x its offset, .y its index in
+// the active list (when it has assignments).
+__device__ __forceinline__ int4 group_block(const pw_page_table* __restrict__ pt, int layer,
                                             const int32_t* __restrict__ idx, int TK, int k,
                                             int E, const PassOut& po,
                                             int32_t* __restrict__ counts,
@@ -159,7 +162,8 @@ __device__ __forceinline__ void group_block(const pw_page_table* __restrict__ pt
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     const int leader = __ffs(peers) - 1;
     int base = 0;
-    for (int w = 0; w < nw; ++w) {
+    const int nwc = min(nw, (TK - c0 + 31) >> 5);  // warps of this chunk holding assignments
+    for (int w = 0; w < nwc; ++w) {
       if (warp == w && e >= 0 && lane == leader) {
         base = run[e];
         run[e] = base + __popc(peers);
@@ -179,6 +183,7 @@ __device__ __forceinline__ void group_block(const pw_page_table* __restrict__ pt
     po.ptok[pb[e] + r] = a / k;
     po.pnn[pb[e] + r] = (pass_np(cnt[e], r / kPassTokens) << 16) | (r % kPassTokens);
   }
+  return ex;
 }
 
 // The one launch before the grouped FFN.  CTA 0 checks the page table and groups the
@@ -199,17 +204,43 @@ __global__ void __launch_bounds__(kGroupThreads) setup_kernel(
   griddep_wait();  // launched as a dependent of whatever precedes it in the stream
   griddep_launch();
   if (blockIdx.x == 0) {
+    // the CUDA-core FFN's per-(module, active expert) block descriptors.  With few experts
+    // (E <= kEarlyDescExperts), thread e reads both blocks of expert e from the page table
+    // before grouping, so those reads overlap it, and files them under e's active index once
+    // the grouping has given it; with many, only the active experts' blocks are read, after it.
+    const bool early = xd != nullptr && E <= kEarlyDescExperts;
+    const bool want_xd = early && static_cast<int>(threadIdx.x) < E;
+    const bool table_ok = pt->blocks != nullptr && static_cast<unsigned>(layer) < pt->num_layers &&
+                          static_cast<int>(pt->num_experts) == E &&
+                          (reinterpret_cast<uintptr_t>(pt->blocks) & 63) == 0;
+    k4::ExpertDesc xg, xdn;
+    if (want_xd && table_ok) {
+      xg = k4::expert_desc(pt, layer, E, threadIdx.x, k4::MODE_GATE_UP, 2 * I, H, 0, 0);
+      xdn = k4::expert_desc(pt, layer, E, threadIdx.x, k4::MODE_DOWN, H, I, 0, 0);
+    }
     for (int e = threadIdx.x; e < E; e += blockDim.x) done[e] = 0;
-    group_block(pt, layer, idx, T * k, k, E, po, counts, offsets, perm, inv, active, meta);
-    if (xd) {  // the CUDA-core FFN's per-(module, active expert) block descriptors
-      __syncthreads();
-      const int na = meta[0];
-      for (int i = threadIdx.x; i < 2 * na; i += blockDim.x) {
-        const int mode = i / na, a = i - mode * na;
-        const int e = active[a];
-        const int rows = mode == k4::MODE_GATE_UP ? 2 * I : H;
-        const int cols = mode == k4::MODE_GATE_UP ? H : I;
-        xd[mode * E + a] = k4::expert_desc(pt, layer, E, e, mode, rows, cols, counts[e], offsets[e]);
+    const int4 ex = group_block(pt, layer, idx, T * k, k, E, po, counts, offsets, perm, inv,
+                                active, meta);
+    if (xd != nullptr) {
+      __syncthreads();  // the grouping's outputs are written (the whole CTA takes the barrier)
+      if (early) {
+        const int c = want_xd && table_ok ? counts[threadIdx.x] : 0;
+        if (c > 0) {
+          xg.te = xdn.te = c;
+          xg.pos0 = xdn.pos0 = ex.x;
+          xd[k4::MODE_GATE_UP * E + ex.y] = xg;
+          xd[k4::MODE_DOWN * E + ex.y] = xdn;
+        }
+      } else {
+        const int na = meta[0];
+        for (int i = threadIdx.x; i < 2 * na; i += blockDim.x) {
+          const int mode = i / na, a = i - mode * na;
+          const int e = active[a];
+          const int rows = mode == k4::MODE_GATE_UP ? 2 * I : H;
+          const int cols = mode == k4::MODE_GATE_UP ? H : I;
+          xd[mode * E + a] =
+              k4::expert_desc(pt, layer, E, e, mode, rows, cols, counts[e], offsets[e]);
+        }
       }
     }
     return;
