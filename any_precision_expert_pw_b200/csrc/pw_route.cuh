@@ -333,6 +333,7 @@ __global__ void __launch_bounds__(256) substitute_kernel(
 }
 
 constexpr int kRemapMaxAssign = 8192;  // T * k of the single-CTA batch rewrites
+constexpr int kRemapGateSmem = 4096;   // up to this T * k the gates are staged in shared memory
 
 // Number of distinct experts among the TK assignments (idx_s: shared copy, or idx: global,
 // read after the CTA's own writes); `flags` [E] and `n` are shared scratch.  CTA-wide: every
@@ -364,6 +365,7 @@ __global__ void __launch_bounds__(1024) remap_kernel(const float* __restrict__ l
   __shared__ uint8_t crit[PW_MAX_EXPERTS];
   __shared__ uint8_t used[PW_MAX_EXPERTS];
   __shared__ int16_t idx_s[kRemapMaxAssign];  // the assignments, scanned once per expert
+  __shared__ float gate_s[kRemapGateSmem];     // their gates (small batches)
   __shared__ int n_r0;
   __shared__ int n_used;
   __shared__ int bad;
@@ -375,10 +377,12 @@ __global__ void __launch_bounds__(1024) remap_kernel(const float* __restrict__ l
   }
   for (int e = tid; e < E; e += blockDim.x) r0[e] = 0;
   __syncthreads();
+  const bool stage_gates = TK <= kRemapGateSmem;
   for (int a = tid; a < TK; a += blockDim.x) {
     const int e = idx[a];
     if (e < 0 || e >= E) atomicExch(&bad, 1);
     idx_s[a] = static_cast<int16_t>(e);
+    if (stage_gates) gate_s[a] = gate[a];
   }
   __syncthreads();
   if (bad) {
@@ -387,11 +391,13 @@ __global__ void __launch_bounds__(1024) remap_kernel(const float* __restrict__ l
   }
   const int before = unique ? distinct_experts(idx_s, nullptr, TK, E, used, &n_used) : 0;
   for (int t = tid; t < T; t += blockDim.x) r0[idx_s[t * k]] = 1;
-  // S_e: float64, ascending (token, slot) order -- one thread per expert scans the batch.
+  // S_e: float64, ascending (token, slot) order -- one thread per expert scans the batch (the
+  // gates from shared memory when staged, so the scan waits on no global load)
+  const float* gsrc = stage_gates ? gate_s : gate;
   for (int e = tid; e < E; e += blockDim.x) {
     double s = 0.0;
     for (int a = 0; a < TK; ++a)
-      if (idx_s[a] == e) s += static_cast<double>(gate[a]);
+      if (idx_s[a] == e) s += static_cast<double>(gsrc[a]);
     S[e] = s;
   }
   __syncthreads();
@@ -463,6 +469,7 @@ __global__ void __launch_bounds__(1024) affinity_remap_kernel(
   __shared__ uint8_t used[PW_MAX_EXPERTS];
   __shared__ uint8_t bin_s[PW_MAX_TOKENS];
   __shared__ int16_t idx_s[kRemapMaxAssign];
+  __shared__ float gate_s[kRemapGateSmem];  // the gates (small batches)
   __shared__ int n_r0;
   __shared__ int n_used;
   __shared__ int bad;
@@ -474,10 +481,12 @@ __global__ void __launch_bounds__(1024) affinity_remap_kernel(
   }
   for (int e = tid; e < E; e += blockDim.x) r0[e] = 0;
   __syncthreads();
+  const bool stage_gates = TK <= kRemapGateSmem;
   for (int a = tid; a < TK; a += blockDim.x) {
     const int e = idx[a];
     if (e < 0 || e >= E) atomicExch(&bad, 1);
     idx_s[a] = static_cast<int16_t>(e);
+    if (stage_gates) gate_s[a] = gate[a];
   }
   __syncthreads();
   if (bad) {
@@ -525,13 +534,15 @@ __global__ void __launch_bounds__(1024) affinity_remap_kernel(
   }
   for (int t = tid; t < T; t += blockDim.x) r0[idx_s[t * k]] = 1;
   __syncthreads();
-  // S_e: one thread per expert scans the batch in (token, slot) order
+  // S_e: one thread per expert scans the batch in (token, slot) order (the gates from shared
+  // memory when staged)
+  const float* gsrc = stage_gates ? gate_s : gate;
   for (int e = tid; e < E; e += blockDim.x) {
     double sc = 0.0;
     for (int t = 0, a = 0; t < T; ++t) {
       const double wt = ldexp(1.0, bin_s[t]);
       for (int s = 0; s < k; ++s, ++a)
-        if (idx_s[a] == e) sc += wt * static_cast<double>(gate[a]);
+        if (idx_s[a] == e) sc += wt * static_cast<double>(gsrc[a]);
     }
     S[e] = sc;
   }
