@@ -428,7 +428,7 @@ __global__ void __launch_bounds__(1024) remap_kernel(const float* __restrict__ l
   }
   for (int t = warp; t < T; t += nw) {
     int cur[PW_MAX_TOPK];
-    for (int j = 0; j < k; ++j) cur[j] = idx[static_cast<size_t>(t) * k + j];
+    for (int j = 0; j < k; ++j) cur[j] = idx_s[t * k + j];  // the staged copy: no global load
     WarpRow<PL> row;
     load_row(logits + static_cast<size_t>(t) * E, E, row);
     uint32_t chosen = lane_set(cur, k);
@@ -574,7 +574,7 @@ __global__ void __launch_bounds__(1024) affinity_remap_kernel(
   for (int t = warp; t < T; t += nw) {
     if (bin_s[t] >= low) continue;  // high-affinity token: its experts stay
     int cur[PW_MAX_TOPK];
-    for (int j = 0; j < k; ++j) cur[j] = idx[static_cast<size_t>(t) * k + j];
+    for (int j = 0; j < k; ++j) cur[j] = idx_s[t * k + j];  // the staged copy: no global load
     WarpRow<PL> row;
     load_row(logits + static_cast<size_t>(t) * E, E, row);
     uint32_t chosen = lane_set(cur, k);
