@@ -306,11 +306,12 @@ size_t pw_moe_workspace_bytes(int T, int k, int E, int H, int I);
  *   contribution is zero).  H % 128 == 0, I % 128 == 0.
  *   Two FFN paths give the same result within the tolerance of the arithmetic (the choice
  *   never changes routing): while T*k < m * min(E, T*k) (m = pw_set_tc_min_tokens, default
- *   4) a CUDA-core bit-plane GEMV in fp32 (each weight decoded once per four tokens);
- *   otherwise the tensor-core GEMM (tcgen05, fp16 operands, fp32 accumulation; each weight
- *   decoded once per 64 tokens of its expert).  On the tensor-core path the activations are
- *   rounded to fp16 (exact for bf16 values within fp16's normal range) and so is h = SiLU(g)
- *   * u; values beyond fp16's range (|v| > 65504) become infinities there.
+ *   4) a CUDA-core bit-plane GEMV (each weight decoded once per four tokens); otherwise the
+ *   tensor-core GEMM (tcgen05; each weight decoded once per 64 tokens of its expert).  Both
+ *   multiply the fp16 LUT values by fp16 activations with fp32 accumulation: x is rounded bf16
+ *   -> fp16 (exact for values within fp16's normal range), h = SiLU(g) * u (computed in fp32)
+ *   is carried as two fp16 parts hi = fp16(h), lo = fp16(h - hi), both multiplied (about 22
+ *   bits of h); values beyond fp16's range (|v| > 65504) become infinities.
  * ------------------------------------------------------------------------------------- */
 pw_status pw_moe_anyprec_forward(const pw_page_table* pt_dev, int layer, int E,
                                  const uint16_t* x_bf16, int T, int H, int I, int k,
