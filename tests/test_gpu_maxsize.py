@@ -1,5 +1,5 @@
-"""Maximum sizes.  The largest batch the forward takes: T = PW_MAX_TOKENS tokens of the tiny layer at top-2, i.e.
-T * k = 8192 assignments, the grouping's limit.  Both FFN paths (the tensor-core GEMM chosen by
+"""Maximum sizes.  The largest batch the forward takes: T = PW_MAX_TOKENS tokens of the tiny
+layer at top-2, i.e. T * k = 8192 assignments, the grouping's limit.  Both FFN paths (the tensor-core GEMM chosen by
 default at 1024 tokens per expert, and the CUDA-core GEMV forced), the grouping read back from
 the workspace bit-exact against the oracle's, and the whole [T, H] output against the float64
 oracle.  One assignment more is refused on the host.  And the largest expert count
