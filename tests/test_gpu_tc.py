@@ -2,8 +2,9 @@
 accumulation) against the CPU oracle, through the C ABI.  The path is forced with
 pw_set_tc_min_tokens(0); the bar is the FFN bar, max |err| <= 2e-3 * rms(y).  Cases: padded
 passes (batches that are not multiples of 16 tokens per expert), several passes of 64 tokens
-per expert, every bitwidth 3..8, ragged stages (H or I not a multiple of 1024), k-sliced down
-projection, experts without tokens, a non-resident block, and the plain path on the same input.
+per expert, every bitwidth 3..8, ragged ends (H or I not a multiple of the 512-column stage or
+the 256-column chunk), k-sliced down projection, experts without tokens, a non-resident block,
+and the plain path on the same input.
 """
 import numpy as np
 import pytest
